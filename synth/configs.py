@@ -1,0 +1,77 @@
+"""The workloads: a dense MXFP4 linear layer and four routed-expert MoE layers.
+
+Dimensions, formats and input distributions follow the five benchmark
+workloads of the FP4 block-scaled MoE study; ``small`` variants keep each
+layer's structure (format, skew, outliers) at sizes a plain CPU reference
+finishes in seconds while still spanning several kernel tiles and a ragged
+tail of expert loads.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+SEED = 0
+SIGMA = 0.02
+
+# tensor ids: the second Philox key word of each weight tensor
+TID_LINEAR = 1
+TID_GATE_UP = 2
+TID_DOWN = 3
+
+
+@dataclass(frozen=True)
+class LinearConfig:
+    name: str
+    fmt: str          # "mxfp4" | "nvfp4"
+    T: int
+    N: int
+    K: int
+    seed: int = SEED
+    sigma: float = SIGMA
+
+    kind = "linear"
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    name: str
+    fmt: str          # "mxfp4" | "nvfp4" | "cb4"
+    T: int
+    E: int
+    H: int
+    I: int
+    k: int
+    zipf_bias: bool = False
+    # planted outliers: (fraction, lo_sigma, hi_sigma) or None
+    outliers: tuple | None = None
+    # CB4 only: absolute outlier threshold for the sparse term
+    cb4_threshold_sigma: float = 6.0
+    swiglu_limit: float = 7.0
+    seed: int = SEED
+    sigma: float = SIGMA
+
+    kind = "moe"
+
+
+LINEAR_C1 = LinearConfig("linear_mxfp4_t16_n2048_k2048", "mxfp4", T=16, N=2048, K=2048)
+MOE_C2 = MoEConfig("moe_mxfp4_decode_e64_h2048_i768_k8_t16", "mxfp4", T=16, E=64, H=2048, I=768, k=8)
+MOE_C3 = MoEConfig("moe_nvfp4_decode_e256_h6144_i2048_k8_t64_zipf", "nvfp4", T=64, E=256, H=6144,
+                   I=2048, k=8, zipf_bias=True, outliers=(0.003, 10.0, 49.0))
+MOE_C4 = MoEConfig("moe_mxfp4_prefill_e256_h6144_i2048_k8_t8192", "mxfp4", T=8192, E=256, H=6144,
+                   I=2048, k=8)
+# ~0.106% of t4 draws exceed 6 sigma on their own; 0.394% more are planted in [6, 49] sigma
+MOE_C5 = MoEConfig("moe_cb4_decode_e64_h2048_i768_k8_t16", "cb4", T=16, E=64, H=2048, I=768, k=8,
+                   outliers=(0.00394, 6.0, 49.0))
+
+FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5)}
+
+
+def small(cfg):
+    """A reduced copy of ``cfg`` with the same structure, for exhaustive CPU comparison."""
+    if cfg.kind == "linear":
+        return replace(cfg, name=cfg.name + "_small", T=5, N=272, K=384)
+    if cfg.fmt == "cb4":
+        return replace(cfg, name=cfg.name + "_small", T=7, E=8, H=384, I=256, k=3)
+    if cfg.T > 1000:  # prefill-shaped: many tokens per expert
+        return replace(cfg, name=cfg.name + "_small", T=300, E=8, H=512, I=384, k=2)
+    return replace(cfg, name=cfg.name + "_small", T=9, E=16, H=512, I=384, k=4)
