@@ -1,0 +1,369 @@
+"""Benchmark of the routed-expert MoE layer on 4-bit block-scaled weights (B200).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+Default workload: the MXFP4 MoE decode layer (64 experts, hidden 2048, expert
+intermediate 768, top-8 softmax router, 16 bf16 tokens). One step = one full
+layer call (router, gate_up + fused SwiGLU-with-clamp, down, weighted combine)
+on device-resident inputs. Metric: decode HBM GB/s = algorithmic bytes per step
+(the active-bytes rule: codes + scales of every expert the step routes to,
+router weights, x and y) / device time per step.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the layer
+(expert weights are not sharded; "replicas only"), the K timed steps are
+bracketed by a barrier and a device synchronisation on both sides, and the
+slowest rank's time is reported: value = all ranks' bytes / that time.
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import configs as C, draws as D  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=C.MOE_C2.name, choices=sorted(C.FULL))
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def per_expert_bytes(cfg):
+    B = 32 if cfg.fmt == "mxfp4" else 16
+    gu = 2 * cfg.I * cfg.H
+    dn = cfg.H * cfg.I
+    b = (gu + dn) // 2 + (gu + dn) // B
+    if cfg.fmt == "nvfp4":
+        b += 8
+    return b, gu // 2 + gu // B + (4 if cfg.fmt == "nvfp4" else 0)
+
+
+def algorithmic_bytes(cfg, counts, tokens=None):
+    """Active-bytes rule: every routed expert's weight bytes once + router + x + y."""
+    per, _ = per_expert_bytes(cfg)
+    d = int(np.count_nonzero(counts))
+    T = cfg.T if tokens is None else tokens
+    router = cfg.E * cfg.H * 4 + (cfg.E * 4 if cfg.zipf_bias else 0)
+    return d * per + router + 2 * T * cfg.H * 2
+
+
+# ------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------
+# our implementation
+# ------------------------------------------------------------------------------------
+def build_layer(cfg, copies, device):
+    import torch
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from helpers import device_weights
+    weights = [device_weights(cfg, device=device)]
+    for _ in range(copies - 1):
+        w0 = weights[0]
+        clone = {n: (None if getattr(w0, n) is None else getattr(w0, n).clone())
+                 for n in ("gu_codes", "gu_scales", "dn_codes", "dn_scales", "gu_tscale", "dn_tscale")}
+        from fp4_block_scaled_moe_b200 import MoEWeights
+        weights.append(MoEWeights(cfg.fmt, cfg.E, cfg.H, cfg.I, clone["gu_codes"], clone["gu_scales"],
+                                  clone["dn_codes"], clone["dn_scales"], clone["gu_tscale"], clone["dn_tscale"],
+                                  cfg.swiglu_limit))
+    x_bits = D.activations_bf16(cfg.seed, cfg.T, cfg.H)
+    wr = D.router_weights(cfg.seed, cfg.E, cfg.H)
+    bias = D.zipf_bias(cfg.seed, cfg.E) if cfg.zipf_bias else None
+    x = torch.from_numpy(x_bits.view(np.int16)).to(device).view(torch.bfloat16)
+    wr_t = torch.from_numpy(wr).to(device)
+    bias_t = None if bias is None else torch.from_numpy(bias).to(device)
+    return weights, x, wr_t, bias_t, x_bits
+
+
+def run_ours(args, cfg, rank, world):
+    import torch
+    import torch.distributed as dist
+    from fp4_block_scaled_moe_b200 import api
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    per, _ = per_expert_bytes(cfg)
+    bank_bytes = per * cfg.E
+    copies = max(2, int(np.ceil(2 * L2_BYTES / bank_bytes)) + 1) if bank_bytes < 4 * L2_BYTES else 1
+    weights, x, wr, bias, x_bits = build_layer(cfg, copies, device)
+    structs = [w.c_struct() for w in weights]
+    T, k = cfg.T, cfg.k
+    ws_bytes = api.moe_fp4_workspace_size(weights[0], T, k)
+    ws = api.alloc_workspace(ws_bytes, device)
+    y = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=device)
+    route = {"counts": torch.empty(cfg.E, dtype=torch.int32, device=device)}
+    stream = torch.cuda.Stream(device)
+
+    def step(i):
+        api.moe_fp4_forward(weights[i % copies], x, wr, bias, k, workspace=ws, y=y, _struct=structs[i % copies],
+                            route_out=route if i == 0 else None)
+
+    with torch.cuda.stream(stream):
+        step(0)
+    torch.cuda.synchronize()
+    counts = route["counts"].cpu().numpy()
+    bytes_step = algorithmic_bytes(cfg, counts)
+    # one CUDA graph per weight copy (kernel launches replayed without host overhead)
+    graphs = []
+    for c in range(copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            step(c)                       # warm the launch path for this copy
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                step(c)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        with torch.cuda.stream(stream):
+            graphs[i % copies].replay()
+    torch.cuda.synchronize()
+    api.fp4_workspace_kernel_stats(ws, reset=True)
+    clk = ClockSampler(device.index if device.index is not None else 0)
+    if not args.no_clocks:
+        clk.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        with torch.cuda.stream(stream):
+            graphs[i % copies].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    clocks = clk.stop() if not args.no_clocks else None
+
+    kern = api.fp4_workspace_kernel_stats(ws)
+
+    # end to end through the C ABI with host buffers: H2D of x, layer, D2H of y each step
+    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for i in range(3):
+        with torch.cuda.stream(stream):
+            x_dev.copy_(x_host, non_blocking=True)
+            api.moe_fp4_forward(weights[i % copies], x_dev, wr, bias, k, workspace=ws, y=y,
+                                _struct=structs[i % copies])
+            y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for i in range(args.steps):
+        with torch.cuda.stream(stream):
+            x_dev.copy_(x_host, non_blocking=True)
+            api.moe_fp4_forward(weights[i % copies], x_dev, wr, bias, k, workspace=ws, y=y,
+                                _struct=structs[i % copies])
+            y_host.copy_(y, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    status = api.fp4_workspace_status(ws)
+
+    gu_ms = kern["gate_up_ns"] / max(kern["gate_up_launches"], 1) / 1e6
+    dn_ms = kern["down_ns"] / max(kern["down_launches"], 1) / 1e6
+    t = torch.tensor([ms_total, e2e_ms, gu_ms, dn_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms, gu_ms, dn_ms = t.tolist()
+    kern_ms = {"gate_up": gu_ms, "down": dn_ms, "launches": kern["gate_up_launches"]}
+    return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, e2e_ms=e2e_ms / args.steps,
+                kern=kern, kern_ms=kern_ms, clocks=clocks, copies=copies, counts=counts, status=status,
+                h2d=T * cfg.H * 2, d2h=T * cfg.H * 2)
+
+
+# ------------------------------------------------------------------------------------
+# reference arm / CPU baseline: the oracle on a bounded sample
+# ------------------------------------------------------------------------------------
+def oracle_sample(cfg, n_tokens):
+    """Quantise (untimed) and return a closure running the oracle layer on n_tokens tokens."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from helpers import LazyOracleBank
+    from oracle import moe as M, routing as R
+    x_bits = D.activations_bf16(cfg.seed, cfg.T, cfg.H)
+    wr = D.router_weights(cfg.seed, cfg.E, cfg.H)
+    bias = D.zipf_bias(cfg.seed, cfg.E) if cfg.zipf_bias else None
+    xf = D.bf16_bits_to_f32(x_bits)
+    tok = np.arange(n_tokens)
+    bank = LazyOracleBank(cfg)
+    lg = R.router_logits(xf[tok], wr, bias)
+    ids = R.topk(lg, cfg.k)
+    for e in np.unique(ids):
+        bank.packed("gu", int(e))
+        bank.packed("dn", int(e))
+    counts = np.bincount(ids.reshape(-1), minlength=cfg.E)
+
+    def run():
+        M.moe_layer(xf[tok], wr, bias, cfg.k, bank, cfg.swiglu_limit)
+
+    return run, algorithmic_bytes(cfg, counts, tokens=n_tokens)
+
+
+def roofline(cfg, r, hbm_peak, peaks):
+    """Dominant kernel: gate_up with the fused SwiGLU. Algorithmic bytes per launch =
+    codes + scales of the gate_up rows of every routed expert + the f16 activation rows
+    read once per unit + h written; duration = its device time per launch in the timed region."""
+    _, gu_per_expert = per_expert_bytes(cfg)
+    d = int(np.count_nonzero(r["counts"]))
+    P = cfg.T * cfg.k
+    alg = d * gu_per_expert + cfg.T * cfg.H * 2 + P * cfg.I * 2
+    ms = r["kern_ms"]["gate_up"]
+    ach = alg / (ms * 1e-3) / 1e9 if ms > 0 else None
+    return {"kernel": "decode_kernel<gate_up+swiglu>", "bound": "hbm", "achieved": ach, "peak": hbm_peak,
+            "unit": "GB/s", "frac": (ach / hbm_peak) if ach else None, "traffic": None,
+            "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if "hbm_gbs" in peaks else "fallback",
+            "bytes_per_launch": int(alg), "ms_per_launch": ms, "down_ms_per_launch": r["kern_ms"]["down"],
+            "timer": "device globaltimer per launch, accumulated in the workspace over the timed steps"}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def main():
+    args = parse()
+    cfg = C.FULL[args.config]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    metric = "FP4 MoE layer: decode HBM GB/s (% of peak); prefill TFLOP/s; tokens/s"
+    workload = cfg.name
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n_tok = 1
+        run, sample_bytes = oracle_sample(cfg, n_tok)
+        for _ in range(args.warmup):
+            run()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            run()
+        dt = (time.perf_counter() - t0) / args.steps
+        v = sample_bytes / dt / 1e9
+        line = {"impl": "reference", "metric": metric, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": workload, "sample": f"{n_tok} token(s) of {cfg.T}, all their experts"},
+                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"{n_tok} token(s) of {cfg.T}, float64 numpy oracle"},
+                "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    r = run_ours(args, cfg, rank, world)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    value = r["bytes_step"] * world / (r["ms_per_step"] * 1e-3) / 1e9
+    line = {
+        "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16xe2m1->f32", "data": "synthetic",
+        "config": {"workload": workload, "tokens": cfg.T, "experts": cfg.E, "hidden": cfg.H, "inter": cfg.I,
+                   "top_k": cfg.k, "format": cfg.fmt, "parallelism": f"replicas{world}",
+                   "l2": f"weights rotate over {r['copies']} copies ({r['copies'] * per_expert_bytes(cfg)[0] * cfg.E / 1e6:.0f} MB) > L2",
+                   "distinct_experts": int(np.count_nonzero(r["counts"])),
+                   "bytes_per_step": int(r["bytes_step"]), "pct_of_hbm_peak": 100 * value / world / hbm_peak},
+        "e2e": {"value": r["bytes_step"] * world / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": 6 * args.steps,
+        "roofline": roofline(cfg, r, hbm_peak, peaks),
+        "clocks": r["clocks"],
+        "device_status": r["status"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

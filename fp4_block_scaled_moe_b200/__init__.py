@@ -1,0 +1,19 @@
+"""fp4moe for B200: the routed-expert MoE layer on 4-bit block-scaled weights.
+
+The computation lives in the CUDA library ``libfp4moe.so`` (C ABI, include/fp4moe.h);
+this package only marshals torch tensors into it.
+"""
+from .api import (  # noqa: F401
+    MoEWeights,
+    alloc_workspace,
+    fp4_linear,
+    fp4_pack,
+    fp4_unpack,
+    fp4_workspace_kernel_stats,
+    fp4_workspace_status,
+    moe_fp4_forward,
+    moe_fp4_workspace_size,
+    moe_route,
+)
+
+__version__ = "0.1.0"

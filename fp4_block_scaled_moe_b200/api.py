@@ -1,0 +1,207 @@
+"""Python binding of the fp4moe C ABI (same names as include/fp4moe.h).
+
+PyTorch supplies device memory and the current stream; every computation runs
+in the library's CUDA kernels. Tensors must be CUDA, contiguous, and of the
+dtype each function states.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib as L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, dtype=None, cuda=True):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fmt_code(fmt):
+    return L.FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def fp4_pack(w: torch.Tensor, fmt="mxfp4"):
+    """Quantise w [..., n, k] (float32 or bf16). Returns (codes, scales, tensor_scale or None)."""
+    lib = L.load()
+    f = fmt_code(fmt)
+    _need(w, "w")
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("w must be float32 or bfloat16")
+    *lead, n, k = w.shape
+    batch = 1
+    for d in lead:
+        batch *= d
+    B = L.BLOCK.get(f, 32)
+    codes = torch.empty((*lead, n, max(k // 2, 1)), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((*lead, n, max(k // B, 1)), dtype=torch.uint8, device=w.device)
+    ts = torch.empty(tuple(lead) if lead else (1,), dtype=torch.float32, device=w.device) if f == L.FP4_NVFP4 else None
+    dt = L.FP4_F32 if w.dtype == torch.float32 else L.FP4_BF16
+    L.check("fp4_pack", lib.fp4_pack(f, _ptr(w), dt, batch, n, k, _ptr(codes), _ptr(scales), _ptr(ts),
+                                     _stream(w.device)))
+    return codes, scales, ts
+
+
+def fp4_unpack(codes, scales, tensor_scale=None, fmt="mxfp4", out_dtype=torch.float32):
+    lib = L.load()
+    f = fmt_code(fmt)
+    _need(codes, "codes", torch.uint8)
+    _need(scales, "scales", torch.uint8)
+    *lead, n, k2 = codes.shape
+    batch = 1
+    for d in lead:
+        batch *= d
+    out = torch.empty((*lead, n, k2 * 2), dtype=out_dtype, device=codes.device)
+    dt = L.FP4_F32 if out_dtype == torch.float32 else L.FP4_BF16
+    L.check("fp4_unpack", lib.fp4_unpack(f, _ptr(codes), _ptr(scales), _ptr(tensor_scale), batch, n, k2 * 2,
+                                         _ptr(out), dt, _stream(codes.device)))
+    return out
+
+
+def moe_route(x, router_w, router_bias, k, logits_in=None):
+    """Router. x [T, H] bf16, router_w [E, H] f32. Returns a dict of device tensors."""
+    lib = L.load()
+    if logits_in is not None:
+        _need(logits_in, "logits_in", torch.float32)
+        T, E = logits_in.shape
+        H = x.shape[1] if x is not None else 0
+        dev = logits_in.device
+    else:
+        _need(x, "x", torch.bfloat16)
+        _need(router_w, "router_w", torch.float32)
+        T, H = x.shape
+        E = router_w.shape[0]
+        dev = x.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    out = dict(
+        logits=torch.empty((T, E), dtype=torch.float32, device=dev),
+        topk_ids=torch.empty((T, k), **i32),
+        topk_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+        counts=torch.empty((E,), **i32),
+        offsets=torch.empty((E + 1,), **i32),
+        perm=torch.empty((T * k,), **i32),
+        inv=torch.empty((T * k,), **i32),
+    )
+    L.check("moe_route", lib.moe_route(_ptr(x), _ptr(router_w), _ptr(router_bias), T, H, E, k, _ptr(logits_in),
+                                       _ptr(out["logits"]), _ptr(out["topk_ids"]), _ptr(out["topk_w"]),
+                                       _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["perm"]),
+                                       _ptr(out["inv"]), _stream(dev)))
+    return out
+
+
+@dataclass
+class MoEWeights:
+    """Device tensors of one MoE layer (see fp4_moe_weights in include/fp4moe.h)."""
+    fmt: str
+    E: int
+    H: int
+    I: int
+    gu_codes: torch.Tensor
+    gu_scales: torch.Tensor
+    dn_codes: torch.Tensor
+    dn_scales: torch.Tensor
+    gu_tscale: torch.Tensor | None = None
+    dn_tscale: torch.Tensor | None = None
+    swiglu_limit: float = 7.0
+    gu_cb: torch.Tensor | None = None
+    gu_rowptr: torch.Tensor | None = None
+    gu_col: torch.Tensor | None = None
+    gu_val: torch.Tensor | None = None
+    dn_cb: torch.Tensor | None = None
+    dn_rowptr: torch.Tensor | None = None
+    dn_col: torch.Tensor | None = None
+    dn_val: torch.Tensor | None = None
+
+    def c_struct(self):
+        s = L.MoEWeightsC()
+        s.fmt = fmt_code(self.fmt)
+        s.num_experts, s.hidden, s.inter = self.E, self.H, self.I
+        s.swiglu_limit = self.swiglu_limit
+        for name in ("gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales", "dn_tscale", "gu_cb",
+                     "gu_rowptr", "gu_col", "gu_val", "dn_cb", "dn_rowptr", "dn_col", "dn_val"):
+            t = getattr(self, name)
+            setattr(s, name, None if t is None else t.data_ptr())
+        return s
+
+
+def moe_fp4_workspace_size(weights: MoEWeights, T: int, k: int) -> int:
+    s = weights.c_struct()
+    return int(L.load().moe_fp4_workspace_size(ctypes.byref(s), T, k))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned device buffer (torch allocations are 512-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def moe_fp4_forward(weights: MoEWeights, x, router_w, router_bias, k, workspace=None, route_out=None,
+                    y=None, _struct=None):
+    """y [T, H] bf16 = MoE layer(x). ``route_out``: optional dict of tensors receiving routing results."""
+    lib = L.load()
+    _need(x, "x", torch.bfloat16)
+    _need(router_w, "router_w", torch.float32)
+    T = x.shape[0]
+    s = _struct if _struct is not None else weights.c_struct()
+    need = int(lib.moe_fp4_workspace_size(ctypes.byref(s), T, k))
+    if workspace is None:
+        if need == 0:
+            raise L.FP4Error("moe_fp4_workspace_size", 1, "invalid layer arguments")
+        workspace = alloc_workspace(need, x.device)
+    if y is None:
+        y = torch.empty((T, weights.H), dtype=torch.bfloat16, device=x.device)
+    ro = None
+    if route_out is not None:
+        ro = L.RouteOutC()
+        for name in ("logits", "topk_ids", "topk_w", "counts", "offsets", "perm", "inv"):
+            t = route_out.get(name)
+            setattr(ro, name, None if t is None else t.data_ptr())
+    L.check("moe_fp4_forward", lib.moe_fp4_forward(ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(router_bias),
+                                                   T, k, _ptr(y), ctypes.byref(ro) if ro is not None else None,
+                                                   _ptr(workspace), workspace.numel(), _stream(x.device)))
+    return y
+
+
+def fp4_linear(x, codes, scales, tensor_scale=None, fmt="mxfp4", workspace=None, y=None):
+    """y [T, N] bf16 = x [T, K] bf16 . W^T with W [N, K] in MXFP4 / NVFP4."""
+    lib = L.load()
+    _need(x, "x", torch.bfloat16)
+    T, K = x.shape
+    N = codes.shape[0]
+    need = int(lib.fp4_linear_workspace_size(T, K))
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    if y is None:
+        y = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    L.check("fp4_linear", lib.fp4_linear(fmt_code(fmt), _ptr(x), T, K, _ptr(codes), _ptr(scales), _ptr(tensor_scale),
+                                         N, _ptr(y), _ptr(workspace), workspace.numel(), _stream(x.device)))
+    return y
+
+
+def fp4_workspace_status(workspace) -> str:
+    code = L.load().fp4_workspace_status(_ptr(workspace), _stream(workspace.device))
+    return L.STATUS.get(code, str(code))
+
+
+def fp4_workspace_kernel_stats(workspace, reset=False) -> dict:
+    """Device time of the grouped expert kernels accumulated in ``workspace`` (see header)."""
+    st = L.KernelStatsC()
+    L.check("fp4_workspace_kernel_stats", L.load().fp4_workspace_kernel_stats(
+        _ptr(workspace), 1 if reset else 0, ctypes.byref(st), _stream(workspace.device)))
+    return {"gate_up_ns": st.gate_up_ns, "gate_up_launches": st.gate_up_launches,
+            "down_ns": st.down_ns, "down_launches": st.down_launches}

@@ -1,0 +1,126 @@
+// C-ABI plumbing: status strings, CUDA error capture, device queries, tensor maps,
+// and the workspace status word.
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace fp4 {
+
+static thread_local char g_last_error[256] = "";
+
+fp4_status record_cuda_error(cudaError_t e, const char* where) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
+                static_cast<int>(e));
+  return FP4_ERR_CUDA;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+fp4_status make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows,
+                           uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                           CUtensorMapSwizzle swz) {
+  auto enc = get_encode();
+  if (enc == nullptr) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return FP4_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {inner_bytes, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return FP4_ERR_CUDA;
+  }
+  return FP4_OK;
+}
+
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" const char* fp4_status_string(fp4_status s) {
+  switch (s) {
+    case FP4_OK: return "FP4_OK";
+    case FP4_ERR_INVALID_ARG: return "FP4_ERR_INVALID_ARG";
+    case FP4_ERR_EMPTY_SHAPE: return "FP4_ERR_EMPTY_SHAPE";
+    case FP4_ERR_SHAPE_OVERFLOW: return "FP4_ERR_SHAPE_OVERFLOW";
+    case FP4_ERR_ALIGNMENT: return "FP4_ERR_ALIGNMENT";
+    case FP4_ERR_UNSUPPORTED: return "FP4_ERR_UNSUPPORTED";
+    case FP4_ERR_WORKSPACE: return "FP4_ERR_WORKSPACE";
+    case FP4_ERR_CUDA: return "FP4_ERR_CUDA";
+    case FP4_ERR_TIMEOUT: return "FP4_ERR_TIMEOUT";
+  }
+  return "FP4_ERR_UNKNOWN";
+}
+
+extern "C" const char* fp4_last_error_string(void) { return g_last_error; }
+
+extern "C" const char* fp4_version(void) { return "0.1.0"; }
+
+extern "C" fp4_status fp4_workspace_status(const void* workspace, void* stream) {
+  if (workspace == nullptr) return FP4_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FP4_TRY_CUDA(cudaStreamSynchronize(st));
+  uint32_t word = 0;
+  FP4_TRY_CUDA(cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost));
+  const uint32_t zero = 0;
+  FP4_TRY_CUDA(cudaMemcpy(const_cast<void*>(workspace), &zero, sizeof(zero), cudaMemcpyHostToDevice));
+  return (word & kStatusTimeout) ? FP4_ERR_TIMEOUT : FP4_OK;
+}
+
+extern "C" fp4_status fp4_workspace_kernel_stats(void* workspace, int reset, fp4_kernel_stats* out, void* stream) {
+  if (workspace == nullptr) return FP4_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FP4_TRY_CUDA(cudaStreamSynchronize(st));
+  WsControl c;
+  FP4_TRY_CUDA(cudaMemcpy(&c, workspace, sizeof(c), cudaMemcpyDeviceToHost));
+  if (out != nullptr) {
+    out->gate_up_ns = c.slot[0].total_ns;
+    out->gate_up_launches = c.slot[0].launches;
+    out->down_ns = c.slot[1].total_ns;
+    out->down_launches = c.slot[1].launches;
+  }
+  if (reset) {
+    for (int i = 0; i < 2; ++i) {
+      c.slot[i].total_ns = 0ull;
+      c.slot[i].launches = 0ull;
+      c.slot[i].start_min = ~0ull;
+      c.slot[i].end_max = 0ull;
+      c.slot[i].done = 0u;
+    }
+    FP4_TRY_CUDA(cudaMemcpy(workspace, &c, sizeof(c), cudaMemcpyHostToDevice));
+  }
+  return FP4_OK;
+}

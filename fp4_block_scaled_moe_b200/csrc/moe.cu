@@ -1,0 +1,236 @@
+// moe_fp4_forward and fp4_linear: argument checks, workspace layout, launch sequence.
+//
+// Layer definition: router top-k ("The gate that missed by 0.0202 pp", section "A file
+// is a census; a decode step is a sample"), experts with the SwiGLU gate and its clamp
+// ("GLM-5.3-Flash-MXFP4" model card, section "Verification compute and EAGLE"), and
+// the gate-weighted sum over the k selected experts.
+#include <cmath>
+
+#include "kernels.cuh"
+
+namespace fp4 {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kTokGroupDecode = 16;
+
+struct MoeWs {
+  size_t status, n_units, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, units_a, units_b, h, o,
+      total;
+  int tiles_a, tiles_b;
+  int64_t max_units_a, max_units_b;
+};
+
+bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
+  const int64_t E = w->num_experts, H = w->hidden, I = w->inter;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  L->tiles_a = static_cast<int>(I / 32);
+  L->tiles_b = static_cast<int>(H / 64);
+  const int64_t groups = (P + kTokGroupDecode - 1) / kTokGroupDecode + std::min<int64_t>(E, P);
+  L->max_units_a = groups * L->tiles_a;
+  L->max_units_b = groups * L->tiles_b;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  L->status = take(sizeof(WsControl));
+  L->n_units = take(64);
+  L->logits = take(sizeof(float) * T * E);
+  L->ids = take(sizeof(int32_t) * P);
+  L->gw = take(sizeof(float) * P);
+  L->counts = take(sizeof(int32_t) * E);
+  L->offsets = take(sizeof(int32_t) * (E + 1));
+  L->perm = take(sizeof(int32_t) * P);
+  L->inv = take(sizeof(int32_t) * P);
+  L->sexp = take(sizeof(int32_t) * T);
+  L->x16 = take(sizeof(uint16_t) * T * H);
+  L->units_a = take(sizeof(int4) * L->max_units_a);
+  L->units_b = take(sizeof(int4) * L->max_units_b);
+  L->h = take(sizeof(uint16_t) * P * I);
+  L->o = take(sizeof(float) * P * H);
+  L->total = off;
+  return true;
+}
+
+fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
+  if (w == nullptr) return FP4_ERR_INVALID_ARG;
+  if (w->fmt != FP4_MXFP4 && w->fmt != FP4_NVFP4) {
+    return (w->fmt == FP4_CB4) ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
+  }
+  int64_t n;
+  FP4_TRY(checked_count({w->num_experts, w->hidden, w->inter, T}, &n));
+  if (k <= 0) return FP4_ERR_EMPTY_SHAPE;
+  const int64_t E = w->num_experts, H = w->hidden, I = w->inter;
+  // byte sizes of the largest tensors must not overflow
+  int64_t tmp;
+  FP4_TRY(checked_count({E, 2 * I, H}, &tmp));
+  int64_t P;
+  if (!mul_ok(T, k, &P) || P >= (int64_t(1) << 31)) return FP4_ERR_SHAPE_OVERFLOW;
+  if (!mul_ok(P, H * 4, &tmp) || !mul_ok(static_cast<int64_t>(T) * E, 4, &tmp)) return FP4_ERR_SHAPE_OVERFLOW;
+  if (E * 2 * I >= (int64_t(1) << 31) || E * H >= (int64_t(1) << 31)) return FP4_ERR_SHAPE_OVERFLOW;
+  if (k > E || k > 32 || E > 1024) return FP4_ERR_INVALID_ARG;
+  const int B = (w->fmt == FP4_MXFP4) ? 32 : 16;
+  if (H % B != 0 || I % B != 0) return FP4_ERR_ALIGNMENT;
+  if (H % 256 != 0 || I % 256 != 0) return FP4_ERR_UNSUPPORTED;
+  if (!(w->swiglu_limit > 0.f) || !(w->swiglu_limit <= 128.f)) return FP4_ERR_INVALID_ARG;
+  if (!w->gu_codes || !w->gu_scales || !w->dn_codes || !w->dn_scales) return FP4_ERR_INVALID_ARG;
+  if (w->fmt == FP4_NVFP4 && (!w->gu_tscale || !w->dn_tscale)) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(w->gu_codes) || !aligned16(w->gu_scales) || !aligned16(w->dn_codes) || !aligned16(w->dn_scales))
+    return FP4_ERR_ALIGNMENT;
+  return FP4_OK;
+}
+
+}  // namespace
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" size_t moe_fp4_workspace_size(const fp4_moe_weights* w, int32_t T, int32_t k) {
+  if (check_moe(w, T, k) != FP4_OK) return 0;
+  MoeWs L;
+  moe_ws_layout(w, T, k, &L);
+  return L.total;
+}
+
+extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
+                                      const float* router_bias, int32_t T, int32_t k, void* y_bf16,
+                                      const fp4_route_out* route, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  FP4_TRY(check_moe(w, T, k));
+  if (!x_bf16 || !router_w || !y_bf16) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(router_w) || !aligned16(y_bf16)) return FP4_ERR_ALIGNMENT;
+  MoeWs L;
+  moe_ws_layout(w, T, k, &L);
+  if (workspace == nullptr || ws_bytes < L.total) return FP4_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return FP4_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = w->num_experts, H = w->hidden, I = w->inter;
+  const int P = T * k;
+
+  auto pick = [](auto* user, void* fallback) { return user ? user : reinterpret_cast<decltype(user)>(fallback); };
+  const fp4_route_out none = {};
+  const fp4_route_out& ro = route ? *route : none;
+  RouteArgs ra{};
+  ra.x = x_bf16; ra.router_w = router_w; ra.router_bias = router_bias;
+  ra.T = T; ra.H = H; ra.E = E; ra.k = k;
+  ra.logits_in = nullptr;
+  ra.logits = pick(ro.logits, ws + L.logits);
+  ra.ids = pick(ro.topk_ids, ws + L.ids);
+  ra.gw = pick(ro.topk_w, ws + L.gw);
+  ra.counts = pick(ro.counts, ws + L.counts);
+  ra.offsets = pick(ro.offsets, ws + L.offsets);
+  ra.perm = pick(ro.perm, ws + L.perm);
+  ra.inv = pick(ro.inv, ws + L.inv);
+  ra.x16 = reinterpret_cast<__half*>(ws + L.x16);
+  ra.sexp = reinterpret_cast<int*>(ws + L.sexp);
+  ra.ctrl = reinterpret_cast<WsControl*>(ws + L.status);
+  ra.wl.units_a = reinterpret_cast<int4*>(ws + L.units_a);
+  ra.wl.units_b = reinterpret_cast<int4*>(ws + L.units_b);
+  ra.wl.tiles_a = L.tiles_a;
+  ra.wl.tiles_b = L.tiles_b;
+  ra.wl.tok_group = kTokGroupDecode;
+  ra.wl.n_units = reinterpret_cast<int*>(ws + L.n_units);
+  ra.pdl_first = true;
+  FP4_TRY(launch_route(ra, st));
+
+  DecodeArgs g{};
+  g.fmt = w->fmt;
+  g.epi = kEpiSwiglu;
+  g.codes = w->gu_codes;
+  g.scales = w->gu_scales;
+  g.tscale = w->gu_tscale;
+  g.rows_total = static_cast<int64_t>(E) * 2 * I;
+  g.K = H;
+  g.rows_per_expert = 2 * I;
+  g.inter = I;
+  g.units = ra.wl.units_a;
+  g.n_units = ra.wl.n_units;
+  g.x16 = ra.x16;
+  g.sexp = ra.sexp;
+  g.perm = ra.perm;
+  g.topk = k;
+  g.gw = ra.gw;
+  g.limit = w->swiglu_limit;
+  g.h_out = reinterpret_cast<__half*>(ws + L.h);
+  g.ldo = I;
+  g.status = &ra.ctrl->status;
+  g.slot = &ra.ctrl->slot[0];
+  FP4_TRY(launch_decode(g, st, true));
+
+  DecodeArgs d = g;
+  d.epi = kEpiDown;
+  d.codes = w->dn_codes;
+  d.scales = w->dn_scales;
+  d.tscale = w->dn_tscale;
+  d.rows_total = static_cast<int64_t>(E) * H;
+  d.K = I;
+  d.rows_per_expert = H;
+  d.units = ra.wl.units_b;
+  d.n_units = ra.wl.n_units + 1;
+  d.x16 = g.h_out;
+  d.sexp = nullptr;
+  d.o_out = reinterpret_cast<float*>(ws + L.o);
+  d.slot = &ra.ctrl->slot[1];
+  d.ldo = H;
+  FP4_TRY(launch_decode(d, st, true));
+
+  const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
+  const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, num_sms() * 8));
+  FP4_TRY(launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, true,
+                     static_cast<const float*>(d.o_out), static_cast<const int32_t*>(ra.inv), T, k, H,
+                     static_cast<uint16_t*>(y_bf16)));
+  (void)P;
+  return FP4_OK;
+}
+
+extern "C" size_t fp4_linear_workspace_size(int32_t T, int64_t K) {
+  if (T <= 0 || K <= 0) return 0;
+  return align_up(256, kAlign) + align_up(sizeof(int32_t) * T, kAlign) +
+         align_up(sizeof(uint16_t) * static_cast<size_t>(T) * static_cast<size_t>(K), kAlign);
+}
+
+extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K,
+                                 const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                                 int64_t N, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return (fmt == FP4_CB4) ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
+  int64_t n;
+  FP4_TRY(checked_count({T, K, N}, &n));
+  int64_t tmp;
+  FP4_TRY(checked_count({N, K}, &tmp));
+  if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 30) || !mul_ok(T, K * 2, &tmp)) return FP4_ERR_SHAPE_OVERFLOW;
+  const int B = (fmt == FP4_MXFP4) ? 32 : 16;
+  if (K % B != 0) return FP4_ERR_ALIGNMENT;
+  if (K % 256 != 0 || N % 64 != 0) return FP4_ERR_UNSUPPORTED;
+  if (!x_bf16 || !codes || !scales || !y_bf16 || (fmt == FP4_NVFP4 && !tensor_scale)) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales) || !aligned16(y_bf16)) return FP4_ERR_ALIGNMENT;
+  const size_t need = fp4_linear_workspace_size(T, K);
+  if (workspace == nullptr || ws_bytes < need) return FP4_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return FP4_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  int* sexp = reinterpret_cast<int*>(ws + 256);
+  __half* x16 = reinterpret_cast<__half*>(ws + 256 + align_up(sizeof(int32_t) * T, kAlign));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, true,
+                     static_cast<const uint16_t*>(x_bf16), static_cast<int>(T), static_cast<int>(K), x16, sexp));
+  DecodeArgs a{};
+  a.fmt = fmt;
+  a.epi = kEpiLinear;
+  a.codes = codes;
+  a.scales = scales;
+  a.tscale = tensor_scale;
+  a.rows_total = N;
+  a.K = static_cast<int>(K);
+  a.rows_per_expert = static_cast<int>(N);
+  a.static_tiles = static_cast<int>(N / 64);
+  a.static_T = T;
+  a.x16 = x16;
+  a.sexp = sexp;
+  a.y_out = static_cast<uint16_t*>(y_bf16);
+  a.ldo = static_cast<int>(N);
+  a.status = status;
+  return launch_decode(a, st, true);
+}

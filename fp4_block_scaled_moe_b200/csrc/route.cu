@@ -1,0 +1,367 @@
+// Router of the MoE layer: logits, top-k with softmax gate weights, per-expert
+// histogram and the stable token permutation; plus the per-expert work lists the
+// grouped expert kernels consume.
+//
+// "The gate that missed by 0.0202 pp", section "A file is a census; a decode step is a
+// sample": a decode step reads the trunk plus the k experts the router picks per token.
+#include <algorithm>
+
+#include "kernels.cuh"
+
+namespace fp4 {
+
+// ---------------------------------------------------------------------------------
+// x (bf16) -> f16 with a per-token power-of-two scale, so that every value fits the
+// f16 range: x16 = x * 2^-s_t with max|x_t| * 2^-s_t in [2^14, 2^15).  One warp per row.
+// ---------------------------------------------------------------------------------
+__device__ void x_row_to_f16(const uint16_t* __restrict__ xrow, int H, __half* __restrict__ out,
+                             int* __restrict__ sexp) {
+  const int lane = threadIdx.x & 31;
+  float amax = 0.f;
+  for (int h = lane * 8; h < H; h += 256) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xrow + h);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  int s = 0;
+  if (amax > 0.f && isfinite(amax)) {
+    int e;
+    frexpf(amax, &e);            // amax = f 2^e, f in [0.5, 1): floor(log2 amax) = e - 1
+    s = (e - 1) - 14;
+  }
+  for (int h = lane * 8; h < H; h += 256) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xrow + h);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half lo = __float2half_rn(ldexpf(__uint_as_float(w[j] << 16), -s));
+      const __half hi = __float2half_rn(ldexpf(__uint_as_float(w[j] & 0xFFFF0000u), -s));
+      o[j] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+    }
+    *reinterpret_cast<uint4*>(out + h) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (lane == 0) *sexp = s;
+}
+
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restrict__ x, int T, int H,
+                                                       __half* __restrict__ x16, int* __restrict__ sexp) {
+  pdl_wait();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row < T) x_row_to_f16(x + static_cast<int64_t>(row) * H, H, x16 + static_cast<int64_t>(row) * H, sexp + row);
+  pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------------
+// R1: logits[t, e] = sum_h x[t, h] w_r[e, h] + bias[e], float32 accumulation.
+// CTA = 8 warps = kExpPerCta experts x (8 / kExpPerCta) warps splitting H, for a group
+// of up to 16 tokens.  CTAs with blockIdx.x == 0 also convert their token rows to f16.
+// ---------------------------------------------------------------------------------
+constexpr int kExpPerCta = 2;
+constexpr int kWarpsPerExp = 8 / kExpPerCta;
+constexpr int kTokGroup = 16;
+
+__global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict__ x,
+                                                     const float* __restrict__ wr,
+                                                     const float* __restrict__ bias, int T, int H, int E,
+                                                     float* __restrict__ logits, __half* __restrict__ x16,
+                                                     int* __restrict__ sexp, WsControl* __restrict__ ctrl) {
+  pdl_wait();
+  if (ctrl != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) {
+    if (threadIdx.x == 0) ctrl->status = 0u;
+    KernelSlot* s = &ctrl->slot[threadIdx.x];
+    s->start_min = ~0ull;
+    s->end_max = 0ull;
+    s->done = 0u;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.y * kTokGroup;
+  const int nt = min(kTokGroup, T - t0);
+  if (x16 != nullptr && blockIdx.x == 0) {
+    for (int r = warp; r < nt; r += 8)
+      x_row_to_f16(x + static_cast<int64_t>(t0 + r) * H, H, x16 + static_cast<int64_t>(t0 + r) * H,
+                   sexp + t0 + r);
+  }
+  const int e = blockIdx.x * kExpPerCta + warp / kWarpsPerExp;
+  const int part = warp % kWarpsPerExp;
+  float acc[kTokGroup];
+#pragma unroll
+  for (int i = 0; i < kTokGroup; ++i) acc[i] = 0.f;
+  if (e < E) {
+    const int hspan = (H / kWarpsPerExp + 7) & ~7;
+    const int h0 = part * hspan, h1 = min(H, h0 + hspan);
+    const float* wrow = wr + static_cast<int64_t>(e) * H;
+    for (int h = h0 + lane * 4; h < h1; h += 128) {
+      const float4 wv = *reinterpret_cast<const float4*>(wrow + h);
+#pragma unroll
+      for (int i = 0; i < kTokGroup; ++i) {
+        if (i < nt) {
+          const uint2 u = *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t0 + i) * H + h);
+          acc[i] = fmaf(__uint_as_float(u.x << 16), wv.x, acc[i]);
+          acc[i] = fmaf(__uint_as_float(u.x & 0xFFFF0000u), wv.y, acc[i]);
+          acc[i] = fmaf(__uint_as_float(u.y << 16), wv.z, acc[i]);
+          acc[i] = fmaf(__uint_as_float(u.y & 0xFFFF0000u), wv.w, acc[i]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kTokGroup; ++i)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
+  __shared__ float part_sum[8][kTokGroup];
+  if (lane == 0)
+#pragma unroll
+    for (int i = 0; i < kTokGroup; ++i) part_sum[warp][i] = acc[i];
+  __syncthreads();
+  if (threadIdx.x < kExpPerCta * kTokGroup) {
+    const int le = threadIdx.x / kTokGroup, i = threadIdx.x % kTokGroup;
+    const int ee = blockIdx.x * kExpPerCta + le;
+    if (ee < E && i < nt) {
+      float s = 0.f;
+      for (int p = 0; p < kWarpsPerExp; ++p) s += part_sum[le * kWarpsPerExp + p][i];
+      if (bias) s += bias[ee];
+      logits[static_cast<int64_t>(t0 + i) * E + ee] = s;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------------
+// R2: top-k per token (one warp per token) and softmax over the selected logits.
+// Order key: larger logit first; equal logits -> lower expert; NaN below every number.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 0u;
+  v = v + 0.0f;                                    // -0 -> +0
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+constexpr int kMaxE = 1024;
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                   int32_t* __restrict__ ids, float* __restrict__ gw) {
+  pdl_wait();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t < T) {
+    const float* lg = logits + static_cast<int64_t>(t) * E;
+    uint32_t key[kMaxE / 32];
+    const int per = (E + 31) / 32;
+#pragma unroll
+    for (int j = 0; j < kMaxE / 32; ++j) {
+      const int e = j * 32 + lane;
+      key[j] = (j < per && e < E) ? order_key(lg[e]) : 0u;
+    }
+    uint32_t taken = 0;   // bit j: my entry j already selected (or absent)
+#pragma unroll
+    for (int j = 0; j < kMaxE / 32; ++j)
+      if (!(j < per && j * 32 + lane < E)) taken |= 1u << j;
+    float sel_logit[32];
+    int sel_id[32];
+    for (int r = 0; r < k; ++r) {
+      uint32_t best = 0;
+      int best_e = 0x7FFFFFFF;
+#pragma unroll
+      for (int j = 0; j < kMaxE / 32; ++j) {
+        if (!(taken >> j & 1u)) {
+          const int e = j * 32 + lane;
+          if (key[j] > best || (key[j] == best && e < best_e)) { best = key[j]; best_e = e; }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int oe = __shfl_xor_sync(0xFFFFFFFFu, best_e, o);
+        if (ob > best || (ob == best && oe < best_e)) { best = ob; best_e = oe; }
+      }
+      if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
+      sel_id[r] = best_e;
+      sel_logit[r] = lg[best_e];
+    }
+    if (lane == 0) {
+      const float m = sel_logit[0];
+      float z[32];
+      float sum = 0.f;
+      for (int r = 0; r < k; ++r) { z[r] = expf(sel_logit[r] - m); sum += z[r]; }
+      for (int r = 0; r < k; ++r) {
+        ids[static_cast<int64_t>(t) * k + r] = sel_id[r];
+        gw[static_cast<int64_t>(t) * k + r] = z[r] / sum;
+      }
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------------
+// R3: counts, offsets, stable permutation and inverse; optional work lists.
+// One CTA of 1024 threads.  Warp w owns the contiguous pair chunk [w C, (w+1) C); the
+// per-warp histograms give each warp its starting cursor per expert, and inside a warp
+// pairs are placed in ascending order with a match/rank step, which keeps the sort stable.
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) perm_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                    int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                    WorkListSpec wl) {
+  extern __shared__ int32_t sm[];
+  int32_t* hist = sm;                       // [32][E]
+  int32_t* off = hist + 32 * E;             // [E + 1]
+  int32_t* scan = off + E + 1;              // [1024] block scan scratch
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 32 * E; i += 1024) hist[i] = 0;
+  __syncthreads();
+  const int C = (P + 31) / 32;
+  const int c0 = warp * C, c1 = min(P, c0 + C);
+  for (int p = c0 + lane; p < c1; p += 32) atomicAdd(&hist[warp * E + ids[p]], 1);
+  __syncthreads();
+  // per expert: exclusive scan over warps, and total count
+  int my_count = 0;
+  for (int e = threadIdx.x; e < E; e += 1024) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int h = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += h;
+    }
+    counts[e] = run;
+    if (e == static_cast<int>(threadIdx.x)) my_count = run;
+  }
+  // exclusive scan of counts over experts (E <= 1024: one value per thread)
+  const int v = (static_cast<int>(threadIdx.x) < E) ? my_count : 0;
+  scan[threadIdx.x] = v;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int add = (static_cast<int>(threadIdx.x) >= o) ? scan[threadIdx.x - o] : 0;
+    __syncthreads();
+    scan[threadIdx.x] += add;
+    __syncthreads();
+  }
+  if (static_cast<int>(threadIdx.x) < E) {
+    off[threadIdx.x] = scan[threadIdx.x] - v;
+    offsets[threadIdx.x] = scan[threadIdx.x] - v;
+  }
+  if (threadIdx.x == 0) { off[E] = P; offsets[E] = P; }
+  __syncthreads();
+  // cursors: hist[w][e] += off[e]
+  for (int i = threadIdx.x; i < 32 * E; i += 1024) hist[i] += off[i % E];
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = c0; base < c1; base += 32) {
+    const int p = base + lane;
+    const bool live = p < c1;
+    const int e = live ? ids[p] : -1 - lane;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & lt);
+    int slot = 0;
+    if (live) slot = hist[warp * E + e] + rank;
+    __syncwarp();
+    if (live && rank == 0) hist[warp * E + e] += __popc(peers);
+    __syncwarp();
+    if (live) {
+      perm[slot] = p;
+      inv[p] = slot;
+    }
+  }
+  // work lists: units {e, tile, slot0, ntok} ordered by expert, token group, tile
+  if (wl.units_a != nullptr) {
+    __syncthreads();
+    for (int list = 0; list < 2; ++list) {
+      int4* units = list == 0 ? wl.units_a : wl.units_b;
+      const int tiles = list == 0 ? wl.tiles_a : wl.tiles_b;
+      if (units == nullptr) continue;
+      const int e = threadIdx.x;
+      const int n = (e < E) ? (off[e + 1] - off[e]) : 0;
+      const int groups = (n + wl.tok_group - 1) / wl.tok_group;
+      const int cnt = groups * tiles;
+      scan[threadIdx.x] = cnt;
+      __syncthreads();
+      for (int o = 1; o < 1024; o <<= 1) {
+        const int add = (static_cast<int>(threadIdx.x) >= o) ? scan[threadIdx.x - o] : 0;
+        __syncthreads();
+        scan[threadIdx.x] += add;
+        __syncthreads();
+      }
+      int u = scan[threadIdx.x] - cnt;
+      if (threadIdx.x == 1023) wl.n_units[list] = scan[1023];
+      for (int g = 0; g < groups; ++g) {
+        const int s0 = off[e] + g * wl.tok_group;
+        const int nt = min(wl.tok_group, n - g * wl.tok_group);
+        for (int tl = 0; tl < tiles; ++tl) units[u++] = make_int4(e, tl, s0, nt);
+      }
+      __syncthreads();
+    }
+  }
+  pdl_launch_dependents();
+}
+
+size_t perm_smem_bytes(int E) { return (32 * static_cast<size_t>(E) + E + 1 + 1024) * sizeof(int32_t); }
+
+fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
+  const int P = a.T * a.k;
+  if (a.logits_in == nullptr) {
+    dim3 grid((a.E + kExpPerCta - 1) / kExpPerCta, (a.T + kTokGroup - 1) / kTokGroup);
+    FP4_TRY(launch_pdl(logits_kernel, grid, dim3(256), 0, st, a.pdl_first,
+                       static_cast<const uint16_t*>(a.x), a.router_w, a.router_bias, a.T, a.H, a.E,
+                       a.logits, a.x16, a.sexp, a.ctrl));
+  } else if (a.x16 != nullptr) {
+    FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((a.T + 7) / 8), dim3(256), 0, st, a.pdl_first,
+                       static_cast<const uint16_t*>(a.x), a.T, a.H, a.x16, a.sexp));
+  }
+  const float* lg = a.logits_in ? a.logits_in : a.logits;
+  FP4_TRY(launch_pdl(topk_kernel, dim3((a.T + 7) / 8), dim3(256), 0, st, true, lg, a.T, a.E, a.k,
+                     a.ids, a.gw));
+  const size_t smem = perm_smem_bytes(a.E);
+  static thread_local int configured_e = -1;
+  if (smem > 48 * 1024 && configured_e < a.E) {
+    FP4_TRY_CUDA(cudaFuncSetAttribute(perm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(perm_smem_bytes(kMaxE))));
+    configured_e = kMaxE;
+  }
+  FP4_TRY(launch_pdl(perm_kernel, dim3(1), dim3(1024), smem, st, true, a.ids, P, a.E, a.counts,
+                     a.offsets, a.perm, a.inv, a.wl));
+  return FP4_OK;
+}
+
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" fp4_status moe_route(const void* x_bf16, const float* router_w, const float* router_bias,
+                                int32_t T, int32_t H, int32_t E, int32_t k, const float* logits_in,
+                                float* logits_out, int32_t* topk_ids, float* topk_w, int32_t* counts,
+                                int32_t* offsets, int32_t* perm, int32_t* inv, void* stream) {
+  int64_t n;
+  FP4_TRY(checked_count({T, E}, &n));
+  if (k <= 0) return FP4_ERR_EMPTY_SHAPE;
+  if (logits_in == nullptr) FP4_TRY(checked_count({T, H, E}, &n));
+  int64_t P;
+  if (!mul_ok(T, k, &P) || P >= (int64_t(1) << 31)) return FP4_ERR_SHAPE_OVERFLOW;
+  if (k > E || k > 32 || E > kMaxE) return FP4_ERR_INVALID_ARG;
+  if (!topk_ids || !topk_w || !counts || !offsets || !perm || !inv) return FP4_ERR_INVALID_ARG;
+  if (logits_in == nullptr) {
+    if (!x_bf16 || !router_w) return FP4_ERR_INVALID_ARG;
+    if (H % 8 != 0) return FP4_ERR_ALIGNMENT;
+    if (!aligned16(x_bf16) || !aligned16(router_w)) return FP4_ERR_ALIGNMENT;
+    if (logits_out == nullptr) return FP4_ERR_INVALID_ARG;   // R1 needs somewhere to write
+  }
+  RouteArgs a{};
+  a.x = x_bf16; a.router_w = router_w; a.router_bias = router_bias;
+  a.T = T; a.H = H; a.E = E; a.k = k;
+  a.logits_in = logits_in; a.logits = logits_out;
+  a.ids = topk_ids; a.gw = topk_w; a.counts = counts; a.offsets = offsets; a.perm = perm; a.inv = inv;
+  a.pdl_first = false;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FP4_TRY(launch_route(a, st));
+  if (logits_in != nullptr && logits_out != nullptr && logits_out != logits_in)
+    FP4_TRY_CUDA(cudaMemcpyAsync(logits_out, logits_in, static_cast<size_t>(T) * E * sizeof(float),
+                                 cudaMemcpyDeviceToDevice, st));
+  return FP4_OK;
+}

@@ -1,0 +1,233 @@
+/*
+ * fp4moe: routed-expert mixture-of-experts layer on 4-bit block-scaled weights,
+ * for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * Formats (defined in "XFP：质量地板驱动的自适应码本量化——3.4 位在双卡工作站跑通 397B MoE",
+ * section 路线二：硬件格式（NVFP4 / MXFP4）):
+ *   MXFP4  E2M1 elements (1 sign, 2 exponent, 1 mantissa bit), 32 per block, one
+ *          UE8M0 power-of-two scale byte per block (value 2^(byte-127); 255 = NaN).
+ *   NVFP4  E2M1 elements, 16 per block, one FP8 E4M3 scale byte per block, times one
+ *          float32 per-tensor ("global") scale.
+ *   CB4    4-bit indices into a 16-entry fp16 codebook per 128-weight group of a row,
+ *          plus a sparse fp16 outlier term in CSR (same page, sections V2, 离群值提取,
+ *          Lloyd 迭代, 子字节打包).
+ * Packing: two 4-bit values per byte, the element with the even index in the low
+ * nibble ("The gate that missed by 0.0202 pp", section "A fused tensor with two
+ * dtypes in it").  Every tensor is row-major and contiguous:
+ *   codes  uint8 [rows, K/2];  scales uint8 [rows, K/B] (B = 32 MXFP4, 16 NVFP4).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device pointers unless stated; the caller allocates and owns
+ *     every buffer, including workspaces.  The library allocates no device memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  Only fp4_workspace_status synchronises.
+ *   - Shapes are checked before any launch with checked 64-bit arithmetic: a zero
+ *     dimension returns FP4_ERR_EMPTY_SHAPE, a width, element count, byte size or
+ *     index that overflows returns FP4_ERR_SHAPE_OVERFLOW ("TensorFold" pull request
+ *     #1050: format classification refuses empty and oversized shapes by name).
+ *     A refused call launches nothing and writes nothing.
+ *   - Device pointers must be 16-byte aligned (FP4_ERR_ALIGNMENT otherwise).
+ *   - CUDA errors are returned as FP4_ERR_CUDA; fp4_last_error_string() has the text.
+ *   - Device-side waits are bounded; one that gives up records FP4_ERR_TIMEOUT in the
+ *     workspace status word and the kernel returns (no trap, no hang).
+ *   - No exceptions cross the ABI.  Entry points are reentrant; concurrent calls
+ *     must not share a workspace.
+ */
+#ifndef FP4MOE_H
+#define FP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef enum fp4_status {
+  FP4_OK = 0,
+  FP4_ERR_INVALID_ARG = 1,    /* null required pointer, bad enum, k > E, k > 32, ... */
+  FP4_ERR_EMPTY_SHAPE = 2,    /* a dimension is zero (or negative) */
+  FP4_ERR_SHAPE_OVERFLOW = 3, /* a derived width / count / byte size overflows */
+  FP4_ERR_ALIGNMENT = 4,      /* K not a multiple of the block, or pointer misaligned */
+  FP4_ERR_UNSUPPORTED = 5,    /* format / size combination this build does not run */
+  FP4_ERR_WORKSPACE = 6,      /* workspace missing or smaller than required */
+  FP4_ERR_CUDA = 7,           /* a CUDA runtime call failed */
+  FP4_ERR_TIMEOUT = 8         /* a bounded device-side wait gave up */
+} fp4_status;
+
+typedef enum fp4_format { FP4_MXFP4 = 1, FP4_NVFP4 = 2, FP4_CB4 = 3 } fp4_format;
+
+typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
+
+/* Human-readable name of a status code (static storage). */
+const char* fp4_status_string(fp4_status s);
+/* Text of the last FP4_ERR_CUDA on the calling thread (static thread-local storage). */
+const char* fp4_last_error_string(void);
+/* Library version, e.g. "0.1.0". */
+const char* fp4_version(void);
+
+/*
+ * fp4_pack: quantise `batch` matrices w [batch, n, k] (float32 or bf16, device) to
+ * MXFP4 or NVFP4.  Outputs: codes [batch, n, k/2], scales [batch, n, k/B] and, for
+ * NVFP4 only, tensor_scale [batch] (float32; one global scale per matrix; pass NULL
+ * for MXFP4).
+ *   MXFP4: per 32-block, e = clamp(floor(log2 amax) - 2, -127, 127) stored as e + 127
+ *          (amax = 0 stores 0); element code = E2M1 round-to-nearest-even of v * 2^-e,
+ *          saturating at 6, sign kept.  A block with a non-finite element stores scale
+ *          0xFF and zero codes.
+ *   NVFP4: ts = amax_tensor / 2688 (1 if amax_tensor = 0); per 16-block
+ *          s = E4M3_rne_satfinite(amax_block / (6 ts)); code = E2M1_rne(v / (s ts)),
+ *          all float32 operations correctly rounded, in that order; a block with s = 0
+ *          stores zero codes; a block with a non-finite element stores scale 0x7F and
+ *          zero codes; the tensor amax ignores non-finite elements.
+ * Requirements: k % B == 0 (FP4_ERR_ALIGNMENT), batch, n, k > 0.
+ * The result is bit-identical to the definition (integer outputs, exact).
+ */
+fp4_status fp4_pack(fp4_format fmt, const void* w, fp4_dtype w_dtype, int64_t batch, int64_t n,
+                    int64_t k, uint8_t* codes, uint8_t* scales, float* tensor_scale, void* stream);
+
+/*
+ * fp4_unpack: inverse of fp4_pack.  out [batch, n, k] (float32 or bf16) receives
+ * E2M1(code) * scale (* tensor_scale for NVFP4), rounded once to the output type
+ * (round to nearest even).  Bit-identical to that definition.
+ */
+fp4_status fp4_unpack(fp4_format fmt, const uint8_t* codes, const uint8_t* scales,
+                      const float* tensor_scale, int64_t batch, int64_t n, int64_t k, void* out,
+                      fp4_dtype out_dtype, void* stream);
+
+/*
+ * moe_route: router of the MoE layer ("The gate that missed by 0.0202 pp", section
+ * "A file is a census; a decode step is a sample": each token reads k of E experts).
+ *   logits[t, e] = sum_h x[t, h] * router_w[e, h] + router_bias[e]   (float32 accumulate)
+ *   topk_ids[t, :] = the k largest logits, descending, ties to the lower expert index
+ *                    (a NaN logit ranks below every number)
+ *   topk_w[t, :]   = softmax over those k logits (float32)
+ *   counts[e]      = number of (t, j) routed to e;  offsets [E+1] = exclusive scan
+ *   perm[slot]     = p = t*k + j, the pairs stably sorted by expert;  inv[p] = slot
+ * x_bf16 [T, H] bf16, router_w [E, H] float32, router_bias [E] or NULL.
+ * logits_in [T, E] (optional): when given, R1 is skipped and these logits are routed,
+ * which makes every output of this call exactly reproducible.  logits_out [T, E] may
+ * be NULL.  All outputs other than logits_out are required.
+ * Requirements: 1 <= k <= min(E, 32), E <= 1024, T * k < 2^31.
+ */
+fp4_status moe_route(const void* x_bf16, const float* router_w, const float* router_bias, int32_t T,
+                     int32_t H, int32_t E, int32_t k, const float* logits_in, float* logits_out,
+                     int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
+                     int32_t* perm, int32_t* inv, void* stream);
+
+/*
+ * Expert weights of one MoE layer: gate_up [E, 2I, H] (rows 0..I-1 gate, I..2I-1 up)
+ * and down [E, H, I], all experts of a matrix fused into one buffer with one stride.
+ *   MXFP4 / NVFP4: *_codes, *_scales as in fp4_pack with batch = E; NVFP4 also
+ *     *_tscale [E] (one global scale per expert matrix); MXFP4 leaves them NULL.
+ *   CB4: *_codes are packed 4-bit indices [E, rows, K/2]; *_cb the fp16 codebooks
+ *     [E, rows, K/128, 16] (uint16 bit patterns); the sparse term is one CSR over the
+ *     E*rows rows of the fused matrix: *_rowptr [E*rows + 1], *_col [nnz] (column in
+ *     the row), *_val [nnz] fp16 bits.  Forward = dense codebook term + sparse term.
+ * swiglu_limit: L of h = silu(min(g, L)) * clamp(u, -L, L), finite, 0 < L <= 128.  Experts
+ *   apply the model's gated SwiGLU together with its clamp ("GLM-5.3-Flash-MXFP4" model
+ *   card, section "Verification compute and EAGLE"); the workload uses L = 7.
+ */
+typedef struct fp4_moe_weights {
+  fp4_format fmt;
+  int32_t num_experts; /* E */
+  int32_t hidden;      /* H */
+  int32_t inter;       /* I */
+  float swiglu_limit;
+  const uint8_t* gu_codes;
+  const uint8_t* gu_scales;
+  const float* gu_tscale;
+  const uint8_t* dn_codes;
+  const uint8_t* dn_scales;
+  const float* dn_tscale;
+  const uint16_t* gu_cb;
+  const int32_t* gu_rowptr;
+  const int32_t* gu_col;
+  const uint16_t* gu_val;
+  const uint16_t* dn_cb;
+  const int32_t* dn_rowptr;
+  const int32_t* dn_col;
+  const uint16_t* dn_val;
+} fp4_moe_weights;
+
+/* Optional copies of the routing results of a forward call (each pointer may be NULL). */
+typedef struct fp4_route_out {
+  float* logits;     /* [T, E] */
+  int32_t* topk_ids; /* [T, k] */
+  float* topk_w;     /* [T, k] */
+  int32_t* counts;   /* [E]    */
+  int32_t* offsets;  /* [E+1]  */
+  int32_t* perm;     /* [T*k]  */
+  int32_t* inv;      /* [T*k]  */
+} fp4_route_out;
+
+/* Bytes of workspace moe_fp4_forward needs for these weights, T tokens and top-k
+ * (0 when the arguments are invalid). */
+size_t moe_fp4_workspace_size(const fp4_moe_weights* w, int32_t T, int32_t k);
+
+/*
+ * moe_fp4_forward: the routed-expert MoE layer.
+ *   route (as moe_route) -> for every routed pair (t, j), e = topk_ids[t, j]:
+ *   [g; u] = W_gu(e) x_t,  h = silu(min(g, L)) * clamp(u, -L, L),  o = W_d(e) h,
+ *   y_t = bf16( sum_{j=0..k-1} topk_w[t, j] * o_{t, j} )   (fixed j order; deterministic)
+ * x_bf16 [T, H], router_w [E, H] float32, router_bias [E] or NULL, y_bf16 [T, H].
+ * workspace: device buffer of at least moe_fp4_workspace_size bytes, 256-byte aligned;
+ * its first 64 bytes hold the status word read by fp4_workspace_status.
+ * route: optional host struct of device pointers receiving the routing results.
+ * Accuracy: float32 accumulation of exactly dequantised weights; against a float64
+ * evaluation of the same definition, rel. Frobenius error <= 5e-3 and per-element
+ * |err| <= 2e-2 (|ref| + 1).
+ */
+fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
+                           const float* router_bias, int32_t T, int32_t k, void* y_bf16,
+                           const fp4_route_out* route, void* workspace, size_t ws_bytes,
+                           void* stream);
+
+/*
+ * fp4_linear: dense W4A16 layer y [T, N] = bf16(x [T, K] . W^T), W [N, K] in MXFP4 or
+ * NVFP4 (codes [N, K/2], scales [N, K/B], tensor_scale [1] for NVFP4, else NULL).
+ * 4-bit weights read with bf16 activations ("TensorFold" pull request #1050,
+ * W4A16_NVFP4).  workspace: at least fp4_linear_workspace_size(T, K) bytes.
+ */
+size_t fp4_linear_workspace_size(int32_t T, int64_t K);
+fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K, const uint8_t* codes,
+                      const uint8_t* scales, const float* tensor_scale, int64_t N, void* y_bf16,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * fp4_workspace_status: synchronise `stream`, then return the status word recorded in
+ * `workspace` by the last call that used it (FP4_OK, or FP4_ERR_TIMEOUT when a bounded
+ * device wait gave up), and clear it.  `workspace` is a device pointer.
+ */
+fp4_status fp4_workspace_status(const void* workspace, void* stream);
+
+/*
+ * Per-kernel device time of the grouped expert kernels, accumulated in the workspace
+ * by the kernels themselves from the device's global nanosecond timer: for each launch,
+ * (last CTA finished) - (first CTA past its dependency wait).  Counters accumulate over
+ * calls that use the same workspace until reset; fp4_workspace_kernel_stats synchronises
+ * `stream`, copies them to *out (host), and zeroes them when `reset` is non-zero.
+ * A freshly allocated workspace must be reset once before its counters mean anything.
+ */
+typedef struct fp4_kernel_stats {
+  uint64_t gate_up_ns;        /* summed device time of the gate_up + SwiGLU kernel */
+  uint64_t gate_up_launches;
+  uint64_t down_ns;           /* summed device time of the down (gate-weighted) kernel */
+  uint64_t down_launches;
+} fp4_kernel_stats;
+
+fp4_status fp4_workspace_kernel_stats(void* workspace, int reset, fp4_kernel_stats* out, void* stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4MOE_H */

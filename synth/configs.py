@@ -69,9 +69,9 @@ FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5)}
 def small(cfg):
     """A reduced copy of ``cfg`` with the same structure, for exhaustive CPU comparison."""
     if cfg.kind == "linear":
-        return replace(cfg, name=cfg.name + "_small", T=5, N=272, K=384)
+        return replace(cfg, name=cfg.name + "_small", T=5, N=320, K=768)
     if cfg.fmt == "cb4":
-        return replace(cfg, name=cfg.name + "_small", T=7, E=8, H=384, I=256, k=3)
+        return replace(cfg, name=cfg.name + "_small", T=7, E=8, H=512, I=256, k=3)
     if cfg.T > 1000:  # prefill-shaped: many tokens per expert
-        return replace(cfg, name=cfg.name + "_small", T=300, E=8, H=512, I=384, k=2)
-    return replace(cfg, name=cfg.name + "_small", T=9, E=16, H=512, I=384, k=4)
+        return replace(cfg, name=cfg.name + "_small", T=300, E=8, H=512, I=256, k=2)
+    return replace(cfg, name=cfg.name + "_small", T=9, E=16, H=768, I=512, k=4)

@@ -102,12 +102,49 @@ def planted_outliers(seed: int, tensor_id: int, start: int, count: int, frac: fl
     return mask, vals
 
 
+_HOST_LIB = None
+
+
+def _host_lib():
+    """The C twin of this recipe (synth/csrc/synth_host.c), or None if it is not built."""
+    global _HOST_LIB
+    if _HOST_LIB is None:
+        import ctypes
+        import os
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp4synth_host.so")
+        if not os.path.exists(path):
+            return None
+        lib = ctypes.CDLL(path)
+        lib.synth_t4_host.restype = None
+        lib.synth_t4_host.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_uint32,
+                                      ctypes.c_uint32, ctypes.c_float, ctypes.c_int, ctypes.c_float,
+                                      ctypes.c_float, ctypes.c_float, ctypes.c_float]
+        _HOST_LIB = lib
+    return _HOST_LIB
+
+
+def expert_weights_c(seed, tensor_id, start, count, sigma=0.02, outliers=None):
+    """Same draws as the numpy path below, computed by the C twin (multi-threaded)."""
+    import ctypes
+    lib = _host_lib()
+    out = np.empty(count, dtype=np.float32)
+    if outliers is None:
+        wo, frac, lo, span = 0, 0.0, 0.0, 0.0
+    else:
+        frac, lo_s, hi_s = outliers
+        wo, frac, lo, span = 1, float(np.float32(frac)), float(np.float32(lo_s)), float(np.float32(hi_s - lo_s))
+    lib.synth_t4_host(out.ctypes.data_as(ctypes.c_void_p), start, count, seed, tensor_id, float(t4_scale(sigma)),
+                      wo, frac, lo, span, float(np.float32(sigma)))
+    return out
+
+
 def expert_weights(seed: int, tensor_id: int, shape, start_row: int = 0, rows: int | None = None,
-                   sigma: float = 0.02, outliers=None) -> np.ndarray:
+                   sigma: float = 0.02, outliers=None, use_c: bool = True) -> np.ndarray:
     """Rows [start_row, start_row + rows) of a weight tensor of ``shape`` (last dim = K).
 
     The tensor is flattened row-major; element i of the flattened tensor is
     drawn from counter i. ``outliers`` is None or (frac, lo_sigma, hi_sigma).
+    ``use_c`` takes the C twin when it is built (identical bits, much faster).
     """
     k = int(shape[-1])
     total_rows = int(np.prod(shape[:-1]))
@@ -116,6 +153,8 @@ def expert_weights(seed: int, tensor_id: int, shape, start_row: int = 0, rows: i
     assert 0 <= start_row and start_row + rows <= total_rows
     start = start_row * k
     count = rows * k
+    if use_c and _host_lib() is not None:
+        return expert_weights_c(seed, tensor_id, start, count, sigma, outliers).reshape(rows, k)
     w = t4_draws(seed, tensor_id, start, count) * t4_scale(sigma)
     if outliers is not None:
         frac, lo_s, hi_s = outliers

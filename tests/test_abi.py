@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every declared symbol, and refuses bad shapes by
+name before touching the device (CPU only; no kernel is launched here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_block_scaled_moe_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "fp4moe.h")
+P = ctypes.c_void_p(0x10000)      # aligned dummy device pointer: never dereferenced on refusal
+PMIS = ctypes.c_void_p(0x10008)   # misaligned
+
+
+def declared():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = "\n".join(l for l in src.splitlines() if not l.lstrip().startswith("#"))
+    return sorted(set(re.findall(r"\b([a-z][a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    lib = L.load()
+    names = declared()
+    assert set(L.SIGNATURES) == set(names), (set(L.SIGNATURES) ^ set(names))
+    for n in names:
+        assert hasattr(lib, n)
+    assert lib.fp4_version() == b"0.1.0"
+    assert lib.fp4_status_string(3) == b"FP4_ERR_SHAPE_OVERFLOW"
+
+
+def _pack(fmt, batch, n, k, w=P, codes=P, scales=P, ts=P):
+    return L.load().fp4_pack(fmt, w, 0, batch, n, k, codes, scales, ts, None)
+
+
+def test_pack_named_refusals():
+    assert _pack(L.FP4_MXFP4, 1, 0, 32) == 2                 # EmptyShape
+    assert _pack(L.FP4_MXFP4, 0, 4, 32) == 2
+    assert _pack(L.FP4_MXFP4, -1, 4, 32) == 2
+    assert _pack(L.FP4_MXFP4, 1 << 40, 1 << 20, 64) == 3     # ShapeOverflow
+    assert _pack(L.FP4_MXFP4, 1, 4, 48) == 4                 # K not a multiple of 32
+    assert _pack(L.FP4_NVFP4, 1, 4, 24) == 4
+    assert _pack(L.FP4_MXFP4, 1, 4, 32, w=PMIS) == 4         # misaligned
+    assert _pack(L.FP4_NVFP4, 1, 4, 32, ts=None) == 1        # NVFP4 needs the tensor scale
+    assert _pack(L.FP4_CB4, 1, 4, 128) == 5
+    assert _pack(9, 1, 4, 32) == 5
+    assert L.load().fp4_unpack(L.FP4_MXFP4, P, P, None, 1, 4, 0, P, 0, None) == 2
+
+
+def test_route_named_refusals():
+    lib = L.load()
+    r = lambda T, H, E, k, lg=None: lib.moe_route(P, P, None, T, H, E, k, lg, P, P, P, P, P, P, P, None)
+    assert r(0, 64, 8, 2) == 2
+    assert r(4, 64, 8, 0) == 2
+    assert r(4, 64, 8, 9) == 1        # k > E
+    assert r(4, 64, 64, 33) == 1      # k > 32
+    assert r(4, 64, 2048, 8) == 1     # E > 1024
+    assert r(4, 60, 8, 2) == 4        # H % 8
+    assert r(1 << 30, 64, 8, 8) == 3  # T k overflows int32
+
+
+def _weights(fmt=L.FP4_MXFP4, E=8, H=512, I=256, lim=7.0):
+    s = L.MoEWeightsC()
+    s.fmt, s.num_experts, s.hidden, s.inter, s.swiglu_limit = fmt, E, H, I, lim
+    for f in ("gu_codes", "gu_scales", "dn_codes", "dn_scales", "gu_tscale", "dn_tscale"):
+        setattr(s, f, 0x10000)
+    return s
+
+
+def test_forward_named_refusals():
+    lib = L.load()
+
+    def fwd(w, T=4, k=2, ws=P, nbytes=1 << 40):
+        return lib.moe_fp4_forward(ctypes.byref(w), P, P, None, T, k, P, None, ws, nbytes, None)
+
+    assert fwd(_weights(E=0)) == 2
+    assert fwd(_weights(), T=0) == 2
+    assert fwd(_weights(H=500)) == 4
+    assert fwd(_weights(H=544)) == 5           # multiple of 32 but not of 256: not run by this build
+    assert fwd(_weights(lim=float("inf"))) == 1
+    assert fwd(_weights(lim=-1.0)) == 1
+    assert fwd(_weights(), k=9) == 1
+    assert fwd(_weights(fmt=L.FP4_CB4)) == 5
+    assert fwd(_weights(E=1 << 20, H=1 << 16, I=1 << 16)) == 3
+    assert fwd(_weights(), ws=None) == 6
+    assert fwd(_weights(), nbytes=100) == 6
+    w = _weights()
+    assert lib.moe_fp4_workspace_size(ctypes.byref(w), 4, 2) > 0
+    assert lib.moe_fp4_workspace_size(ctypes.byref(_weights(E=0)), 4, 2) == 0
+
+
+def test_linear_named_refusals():
+    lib = L.load()
+    lin = lambda fmt, T, K, N, ws=P: lib.fp4_linear(fmt, P, T, K, P, P, P, N, P, ws, 1 << 40, None)
+    assert lin(L.FP4_MXFP4, 0, 256, 64) == 2
+    assert lin(L.FP4_MXFP4, 4, 48, 64) == 4
+    assert lin(L.FP4_MXFP4, 4, 256, 65) == 5
+    assert lin(L.FP4_MXFP4, 4, 1 << 40, 64) == 3
+    assert lin(L.FP4_MXFP4, 4, 256, 64, ws=None) == 6

@@ -59,3 +59,10 @@ def test_configs_dims():
     for c in configs.FULL.values():
         s = configs.small(c)
         assert s.fmt == c.fmt
+
+
+def test_c_twin_equals_numpy():
+    for o in (None, (0.00394, 6.0, 49.0)):
+        a = draws.expert_weights(0, 3, (400, 384), start_row=33, rows=150, outliers=o, use_c=False)
+        b = draws.expert_weights(0, 3, (400, 384), start_row=33, rows=150, outliers=o, use_c=True)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
