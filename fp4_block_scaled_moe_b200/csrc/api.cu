@@ -13,6 +13,7 @@ namespace fp4 {
 static thread_local char g_last_error[256] = "";
 
 fp4_status record_cuda_error(cudaError_t e, const char* where) {
+  (void)cudaGetLastError();   // clear a non-sticky error so the next call starts clean
   std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
                 static_cast<int>(e));
   return FP4_ERR_CUDA;

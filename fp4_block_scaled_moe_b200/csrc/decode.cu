@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 Layout make_layout(int fmt, int K) {
   Layout L{};
   const int B = (fmt == FP4_MXFP4) ? 32 : 16;
-  const int smem_cap = 227 * 1024;
+  const int smem_cap = 227 * 1024 - 256;    // leave room for the kernel's static shared memory
   const int extra = kRows * kOutPitch * 4 + 16 * kMaxStages + 1024;
   for (int kc : {1024, 768, 512, 256}) {
     if (K % kc != 0) continue;
@@ -340,8 +340,8 @@ fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& m
   auto kern = decode_kernel<kFmt, kEpi>;
   static thread_local int configured = 0;
   if (configured < L.smem_bytes) {
-    FP4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    configured = 227 * 1024;
+    FP4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem_bytes));
+    configured = L.smem_bytes;
   }
   return launch_pdl(kern, dim3(grid), dim3(kThreads), static_cast<size_t>(L.smem_bytes), st, pdl, map, a, L);
 }
