@@ -1,33 +1,41 @@
 // Grouped W4A16 GEMV for the decode path: few tokens per expert, so the layer is
 // bound by the weight stream from HBM.
 //
-// Design (B200): a persistent CTA per SM walks a list of work units {expert, 64-row
-// weight tile, up to 16 routed tokens}.  One producer warp streams each unit's 4-bit
-// codes with TMA (128-byte swizzled boxes, conflict-free for the fragment reads), its
-// scale bytes with 4-byte async copies, and the f16 activation rows with 1D bulk copies
-// into a multi-stage shared-memory ring guarded by mbarriers.  Eight consumer warps
-// dequantise in registers (E2M1 pairs -> f16x2 with the sm_100 conversion instruction;
-// NVFP4 E4M3 block scales folded in f16, exact; MXFP4 power-of-two scales applied per
-// 32-block in fp32) and accumulate with warp-level f16 MMAs into fp32.  The two K
-// halves meet in shared memory and a fused epilogue writes: the SwiGLU-with-clamp
-// activation h (gate_up), the gate-weighted expert output (down), or y (dense layer).
+// Design (B200): persistent CTAs, two per SM, walk work units {expert, 64-row weight
+// tile, up to 8 routed tokens}.  One producer warp streams a unit's 4-bit codes with TMA
+// (128-byte swizzled boxes, conflict-free for the fragment reads), its scale bytes with
+// 4-byte async copies and the f16 activation rows with 1D bulk copies into a shared-
+// memory ring guarded by mbarriers.  Eight consumer warps (32 rows x a quarter of the
+// stage's K each) dequantise in registers -- E2M1 pairs -> f16x2 with the sm_100
+// conversion instruction; NVFP4 E4M3 block scales folded into the f16 operand (exact);
+// MXFP4 power-of-two scales applied per 32-block to fp32 partial sums -- and accumulate
+// with warp-level f16 MMAs into fp32.  The four K quarters meet in shared memory in a
+// fixed order and a fused epilogue writes the SwiGLU-with-clamp activation (gate_up),
+// the gate-weighted expert output (down) or y (dense layer).
 //
-// The per-element unpack-and-scale cost is the overhead the MXFP4 campaign measured
-// ("The gate that missed by 0.0202 pp", section "Serving throughput": a constant loss
-// paid once per weight element per step); here it runs in registers beside the stream.
+// In kModeRoute the gate_up kernel also finishes the router in its prologue: every CTA
+// takes the top-k of the logits, the per-expert counts and the stable permutation into
+// shared memory (CTA 0 also stores them for the later kernels), so no separate launch
+// sits between the logits and the weight stream.
+//
+// The per-element unpack-and-scale work is the cost the MXFP4 serving campaign measured
+// as a constant overhead per weight element ("The gate that missed by 0.0202 pp",
+// section "Serving throughput"); here it runs in registers beside the HBM stream.
 #include <algorithm>
 
 #include "kernels.cuh"
+#include "routing.cuh"
 
 namespace fp4 {
 namespace {
 
 constexpr int kRows = 64;                 // weight rows per unit
-constexpr int kTok = 16;                  // tokens per unit
+constexpr int kTok = 8;                   // tokens per unit (one n8 MMA tile)
 constexpr int kConsumers = 8;             // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;
-constexpr int kMaxStages = 4;
-constexpr int kOutPitch = kTok + 1;       // fp32 staging row pitch (bank spread)
+constexpr int kMaxStages = 8;
+constexpr int kRedPitch = kTok + 1;       // fp32 reduction row pitch
+constexpr int kSmemBudget = 110 * 1024;   // two CTAs per SM
 
 struct Layout {
   int kc;            // K elements per stage
@@ -37,7 +45,10 @@ struct Layout {
   int x_row;         // bytes per token row in the stage (padded)
   int stage_bytes;
   int stages;
-  int out_off;       // fp32 staging for the K-half reduction
+  int red_off;       // 2 x [64][kRedPitch] fp32
+  int lut_off;       // 256 fp32 (UE8M0 -> float)
+  int cnt_off, off_off, pre_off;   // [E + 1] int each (pre is followed by [E] cursors)
+  int perm_off;      // [P] int (kModeRoute)
   int bar_off;
   int smem_bytes;
 };
@@ -45,15 +56,29 @@ struct Layout {
 __device__ __forceinline__ void named_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
 }
-
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ float ldsf(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16u(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ uint32_t lds8(uint32_t addr) {
@@ -72,21 +97,64 @@ struct Unit {
   int e, tile, slot0, ntok;
 };
 
-__device__ __forceinline__ Unit load_unit(const DecodeArgs& a, int u) {
-  Unit un;
-  if (a.units != nullptr) {
-    const int4 v = a.units[u];
-    un.e = v.x; un.tile = v.y; un.slot0 = v.z; un.ntok = v.w;
-  } else {
-    un.e = 0;
-    un.tile = u % a.static_tiles;
-    un.slot0 = (u / a.static_tiles) * kTok;
-    un.ntok = min(kTok, a.static_T - un.slot0);
+// Exclusive scans by warp 0 over E experts: off = scan(cnt), pre = scan(units per expert).
+__device__ void scan_experts(const int* cnt, int* off, int* pre, int E, int tiles) {
+  const int lane = threadIdx.x & 31;
+  const int per = (E + 31) / 32;
+  const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+  int sc = 0, su = 0;
+  for (int e = e0; e < e1; ++e) {
+    sc += cnt[e];
+    su += (cnt[e] + kTok - 1) / kTok * tiles;
   }
+  int ic = sc, iu = su;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int vc = __shfl_up_sync(0xFFFFFFFFu, ic, o), vu = __shfl_up_sync(0xFFFFFFFFu, iu, o);
+    if (lane >= o) { ic += vc; iu += vu; }
+  }
+  int rc = ic - sc, ru = iu - su;
+  for (int e = e0; e < e1; ++e) {
+    off[e] = rc;
+    pre[e] = ru;
+    rc += cnt[e];
+    ru += (cnt[e] + kTok - 1) / kTok * tiles;
+  }
+  if (lane == 31) {
+    off[E] = ic;
+    pre[E] = iu;
+  }
+}
+
+// unit u -> {expert, tile, first slot, tokens}; units are ordered by expert, tile, group
+__device__ __forceinline__ Unit unit_of(int u, const int* cnt, const int* off, const int* pre, int E,
+                                        int tiles) {
+  int lo = 0, hi = E - 1;          // largest e with pre[e] <= u
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  Unit un;
+  un.e = lo;
+  const int n = cnt[lo];
+  const int groups = (n + kTok - 1) / kTok;
+  const int local = u - pre[lo];
+  un.tile = local / groups;
+  const int grp = local - un.tile * groups;
+  un.slot0 = off[lo] + grp * kTok;
+  un.ntok = min(kTok, n - grp * kTok);
   return un;
 }
 
-// global weight row of unit row r (0..63)
+__device__ __forceinline__ Unit unit_static(int u, int tiles, int T) {
+  Unit un;
+  un.e = 0;
+  un.tile = u % tiles;
+  un.slot0 = (u / tiles) * kTok;
+  un.ntok = min(kTok, T - un.slot0);
+  return un;
+}
+
 template <int kEpi>
 __device__ __forceinline__ int64_t unit_row(const DecodeArgs& a, const Unit& un, int r) {
   const int64_t base = static_cast<int64_t>(un.e) * a.rows_per_expert;
@@ -95,24 +163,29 @@ __device__ __forceinline__ int64_t unit_row(const DecodeArgs& a, const Unit& un,
   return base + static_cast<int64_t>(un.tile) * kRows + r;
 }
 
-// activation row feeding unit token i
-template <int kEpi>
-__device__ __forceinline__ int x_row_of(const DecodeArgs& a, const Unit& un, int i) {
-  if (kEpi == kEpiSwiglu) return a.perm[un.slot0 + i] / a.topk;
-  return un.slot0 + i;
-}
-
-template <int kFmt, int kEpi>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kFmt, int kEpi, int kMode, int KC>
+__global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a, const Layout L) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // stage geometry (must match make_layout)
+  constexpr int kB = (kFmt == FP4_MXFP4) ? 32 : 16;
+  constexpr int kScaleRow = KC / kB;                 // scale bytes per row per stage
+  constexpr int kScalesOff = kRows * KC / 2;
+  constexpr int kXOff = kScalesOff + kRows * kScaleRow;
+  constexpr int kXRow = 2 * KC + 64;                 // padded f16 token row
+  constexpr int kNq = KC / 128;                      // 32-K regions per warp per stage
+  extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // 128-byte swizzled TMA boxes need 1024-byte aligned destinations
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - smem_u32(smem_raw));
-  const uint32_t bar_full = sbase + L.bar_off;                 // [stages] x 8 bytes
+  const uint32_t bar_full = sbase + L.bar_off;
   const uint32_t bar_empty = bar_full + 8 * kMaxStages;
   constexpr int B = (kFmt == FP4_MXFP4) ? 32 : 16;
+  const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 32 : a.rows_per_expert / kRows;
+  int* cnt = reinterpret_cast<int*>(smem + L.cnt_off);
+  int* off = reinterpret_cast<int*>(smem + L.off_off);
+  int* pre = reinterpret_cast<int*>(smem + L.pre_off);
+  int* perm_s = reinterpret_cast<int*>(smem + L.perm_off);
 
   __shared__ unsigned int exit_count;
   if (threadIdx.x == 0) {
@@ -123,30 +196,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     exit_count = 0u;
   }
+  if (kFmt == FP4_MXFP4)
+    for (int i = threadIdx.x; i < 256; i += kThreads)
+      reinterpret_cast<float*>(smem + L.lut_off)[i] = ue8m0_to_f32(static_cast<uint32_t>(i));
   if (warp == kConsumers && lane == 0) prefetch_tmap(&tmap);
   __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
   if (threadIdx.x == 0) slot_begin(a.slot);
-  // the last warp of the CTA to leave records the CTA's end time
-  auto finish = [&]() {
+  auto finish = [&]() {   // the last warp of the CTA to leave records the CTA's end time
     if (lane == 0 && atomicAdd(&exit_count, 1u) == kConsumers) slot_end(a.slot);
   };
 
-  const int n_units = (a.n_units != nullptr) ? *a.n_units
-                                             : a.static_tiles * ((a.static_T + kTok - 1) / kTok);
-  const int ncb = L.kc / 256;                                  // 128-byte code boxes per row per stage
+  // ------------------------------- work units ---------------------------------------
+  int n_units;
+  if (kMode == kModeStatic) {
+    n_units = tiles * ((a.T + kTok - 1) / kTok);
+  } else {
+    const int E = a.E;
+    if (kMode == kModeRoute) {
+      const int P = a.T * a.topk;
+      int* ids_s = reinterpret_cast<int*>(smem);       // scratch in the (still unused) stage ring
+      for (int t = warp; t < a.T; t += kConsumers + 1)
+        topk_warp(a.logits + static_cast<int64_t>(t) * E, E, a.topk, ids_s + t * a.topk,
+                  blockIdx.x == 0 ? a.gw + static_cast<int64_t>(t) * a.topk : nullptr);
+      for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = 0;
+      __syncthreads();
+      for (int p = threadIdx.x; p < P; p += kThreads) {
+        atomicAdd(&cnt[ids_s[p]], 1);
+        if (blockIdx.x == 0) a.ids[p] = ids_s[p];
+      }
+      __syncthreads();
+      if (warp == 0) {
+        scan_experts(cnt, off, pre, E, tiles);
+        __syncwarp();
+        // stable placement: pairs in ascending order, 32 per round, ranked within the round
+        int* cur = pre + E + 1;                      // [E] cursors
+        for (int e = lane; e < E; e += 32) cur[e] = off[e];
+        __syncwarp();
+        const unsigned lt = (1u << lane) - 1u;
+        for (int base = 0; base < P; base += 32) {
+          const int p = base + lane;
+          const bool live = p < P;
+          const int e = live ? ids_s[p] : -1 - lane;
+          const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+          const int rank = __popc(peers & lt);
+          const int slot = live ? cur[e] + rank : 0;
+          __syncwarp();
+          if (live && rank == 0) cur[e] += __popc(peers);
+          __syncwarp();
+          if (live) {
+            perm_s[slot] = p;
+            if (blockIdx.x == 0) {
+              a.perm[slot] = p;
+              a.inv[p] = slot;
+            }
+          }
+        }
+      }
+      __syncthreads();
+      if (blockIdx.x == 0)
+        for (int e = threadIdx.x; e <= E; e += kThreads) {
+          if (e < E) a.counts[e] = cnt[e];
+          a.offsets[e] = off[e];
+        }
+    } else {
+      for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = a.counts[e];
+      __syncthreads();
+      if (warp == 0) scan_experts(cnt, off, pre, E, tiles);
+      __syncthreads();
+    }
+    n_units = pre[E];
+  }
+  auto get_unit = [&](int u) -> Unit {
+    if (kMode == kModeStatic) return unit_static(u, tiles, a.T);
+    return unit_of(u, cnt, off, pre, a.E, tiles);
+  };
+  auto perm_at = [&](int slot) -> int {
+    if (kMode == kModeRoute) return perm_s[slot];
+    return a.perm[slot];
+  };
+  constexpr int ncb = KC / 256;                                // 128-byte code boxes per row per stage
 
   if (warp == kConsumers) {
     // ------------------------------- producer -------------------------------------
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit un = load_unit(a, u);
+      const Unit un = get_unit(u);
       const int64_t y0 = unit_row<kEpi>(a, un, 0), y1 = unit_row<kEpi>(a, un, 32);
-      const int xr = (lane < un.ntok) ? x_row_of<kEpi>(a, un, lane) : 0;
-      const uint32_t tx = static_cast<uint32_t>(kRows * (L.kc / 2) + un.ntok * L.kc * 2);
-      const int words = L.scale_row / 4;
+      int xr = 0;
+      if (lane < un.ntok) xr = (kEpi == kEpiSwiglu) ? perm_at(un.slot0 + lane) / a.topk : un.slot0 + lane;
+      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2);
+      constexpr int words = kScaleRow / 4;
       for (int c = 0; c < L.nchunks; ++c, ++it) {
         const int s = it % L.stages;
         if (it >= L.stages && !mbar_wait(bar_empty + 8 * s, ((it / L.stages) & 1) ^ 1, a.status)) {
@@ -154,12 +296,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t st_base = sbase + s * L.stage_bytes;
-        const int k0 = c * L.kc;
-        // scale bytes: 64 rows x scale_row, 4-byte async copies
+        const int k0 = c * KC;
         for (int w = lane; w < kRows * words; w += 32) {
-          const int r = w / words, cw = w % words;
+          const int r = w / words, cw = w - r * words;
           const uint8_t* src = a.scales + unit_row<kEpi>(a, un, r) * (a.K / B) + k0 / B + cw * 4;
-          cp_async4(st_base + L.scales_off + r * L.scale_row + cw * 4, src);
+          cp_async4(st_base + kScalesOff + r * kScaleRow + cw * 4, src);
         }
         cp_async_arrive(bar_full + 8 * s);
         __syncwarp();
@@ -167,12 +308,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         for (int q = lane; q < 2 * ncb; q += 32) {
           const int rb = q & 1, cb = q >> 1;
-          tma_load_2d(st_base + L.codes_off + (cb * kRows + rb * 32) * 128, &tmap, k0 / 2 + cb * 128,
+          tma_load_2d(st_base + (cb * kRows + rb * 32) * 128, &tmap, k0 / 2 + cb * 128,
                       static_cast<int32_t>(rb ? y1 : y0), bar_full + 8 * s);
         }
         if (lane < un.ntok)
-          bulk_g2s(st_base + L.x_off + lane * L.x_row, a.x16 + static_cast<int64_t>(xr) * a.K + k0,
-                   static_cast<uint32_t>(L.kc * 2), bar_full + 8 * s);
+          bulk_g2s(st_base + kXOff + lane * kXRow, a.x16 + static_cast<int64_t>(xr) * a.K + k0,
+                   static_cast<uint32_t>(KC * 2), bar_full + 8 * s);
       }
     }
     // drain: never leave while copies into this CTA's shared memory are in flight
@@ -185,21 +326,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // --------------------------------- consumers --------------------------------------
-  const int rg = warp & 3, kh = warp >> 2;
+  const int rh = warp & 1, kq = warp >> 1;
   const int g = lane >> 2, t = lane & 3;
-  const int r0 = rg * 16 + g, r1 = r0 + 8;
-  float* outs = reinterpret_cast<float*>(smem + L.out_off);
-  const int nreg = L.kc / 32;                                  // 32-K regions per stage
-  const int j0 = kh * (nreg / 2), j1 = j0 + nreg / 2;
+  const int rbase = 32 * rh + g;                 // rows rbase + 8m, m = 0..3
+  float* red = reinterpret_cast<float*>(smem + L.red_off);
+  const uint32_t lut = sbase + L.lut_off;
+  const int jbase = kq * kNq;                    // this warp's first 32-K region of a stage
+  // per-thread offsets within a stage: codes (swizzled 128-byte rows), scales, activations
+  const uint32_t c_off = ((jbase >> 3) * kRows + rbase) * 128 + 4 * t;
+  uint32_t c_xo[kNq];
+#pragma unroll
+  for (int jj = 0; jj < kNq; ++jj) c_xo[jj] = static_cast<uint32_t>((((jbase & 7) + jj) ^ g) << 4);
+  const uint32_t s_off = kScalesOff + rbase * kScaleRow + (kFmt == FP4_MXFP4 ? jbase : 2 * jbase);
+  const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
   int it = 0;
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-    const Unit un = load_unit(a, u);
-    const int ntiles = un.ntok > 8 ? 2 : 1;
+    const Unit un = get_unit(u);
     float acc[2][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int m = 0; m < 2; ++m)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+      for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
     for (int c = 0; c < L.nchunks; ++c, ++it) {
       const int s = it % L.stages;
       if (!mbar_wait(bar_full + 8 * s, (it / L.stages) & 1, a.status)) {
@@ -207,99 +354,134 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
       }
       const uint32_t st_base = sbase + s * L.stage_bytes;
-      const uint32_t cbase = st_base + L.codes_off;
-      const uint32_t sc_r0 = st_base + L.scales_off + r0 * L.scale_row;
-      const uint32_t sc_r1 = st_base + L.scales_off + r1 * L.scale_row;
-      const uint32_t xbase = st_base + L.x_off + g * L.x_row + t * 16;
-      for (int j = j0; j < j1; ++j) {
-        const uint32_t box = cbase + ((j >> 3) * kRows) * 128;
-        const uint32_t w0 = lds32(box + r0 * 128 + (((j & 7) ^ (r0 & 7)) << 4) + 4 * t);
-        const uint32_t w1 = lds32(box + r1 * 128 + (((j & 7) ^ (r1 & 7)) << 4) + 4 * t);
-        uint32_t p0[4], p1[4];   // f16x2 of row r0 / r1: bytes 0..3 of the word
-        e2m1x8_to_f16x8(w0, p0[0], p0[1], p0[2], p0[3]);
-        e2m1x8_to_f16x8(w1, p1[0], p1[1], p1[2], p1[3]);
+      // scale bytes of this warp's regions, one load per row
+      uint32_t sb[4][(kFmt == FP4_MXFP4) ? 1 : 2];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t addr = st_base + s_off + m * 8 * kScaleRow;
+        if (kFmt == FP4_MXFP4) {
+          static_assert(kFmt != FP4_MXFP4 || kNq <= 4, "scale word");
+          sb[m][0] = (kNq == 4) ? lds32(addr) : lds16u(addr);
+        } else if (kNq == 4) {
+          const uint2 v = lds64(addr);                 // 2 kNq = 8 bytes
+          sb[m][0] = v.x;
+          sb[m][(kFmt == FP4_MXFP4) ? 0 : 1] = v.y;
+        } else {
+          sb[m][0] = lds32(addr);                      // 2 kNq = 4 bytes
+          sb[m][(kFmt == FP4_MXFP4) ? 0 : 1] = 0u;
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < kNq; ++jj) {
+        const uint32_t caddr = st_base + c_off + c_xo[jj];
+        uint32_t w[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) w[m] = lds32(caddr + m * 8 * 128);
+        uint32_t p[4][4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) e2m1x8_to_f16x8(w[m], p[m][0], p[m][1], p[m][2], p[m][3]);
+        const uint4 xq = lds128(st_base + x_off + jj * 64);
         if (kFmt == FP4_NVFP4) {
-          // this thread's 8 K positions all lie in block 2j + (t >> 1)
-          const int blk = 2 * j + (t >> 1);
-          const uint32_t s01 = e4m3x2_to_f16x2(lds8(sc_r0 + blk) | (lds8(sc_r1 + blk) << 8));
-          const uint32_t s0 = __byte_perm(s01, 0, 0x1010), s1 = __byte_perm(s01, 0, 0x3232);
+          // this thread's 8 K positions lie in block 2j + (t >> 1): byte 2 jj + (t >> 1) of the row's run
+          const int bsel = 2 * jj + (t >> 1);
+          uint32_t b4[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) { p0[q] = hmul2(p0[q], s0); p1[q] = hmul2(p1[q], s1); }
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t word = (bsel < 4) ? sb[m][0] : sb[m][(kFmt == FP4_MXFP4) ? 0 : 1];
+            b4[m] = (word >> (8 * (bsel & 3))) & 0xFFu;
+          }
+          const uint32_t s01 = e4m3x2_to_f16x2(b4[0] | (b4[1] << 8));
+          const uint32_t s23 = e4m3x2_to_f16x2(b4[2] | (b4[3] << 8));
+          const uint32_t sc[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                                  __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
 #pragma unroll
-          for (int tl = 0; tl < 2; ++tl) {
-            if (tl < ntiles) {
-              const uint4 xq = lds128(xbase + tl * 8 * L.x_row + j * 64);
-              mma_16816(acc[tl], p0[0], p1[0], p0[1], p1[1], xq.x, xq.y);
-              mma_16816(acc[tl], p0[2], p1[2], p0[3], p1[3], xq.z, xq.w);
-            }
+          for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) p[m][q] = hmul2(p[m][q], sc[m]);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_16816(acc[mt], p[2 * mt][0], p[2 * mt + 1][0], p[2 * mt][1], p[2 * mt + 1][1], xq.x, xq.y);
+            mma_16816(acc[mt], p[2 * mt][2], p[2 * mt + 1][2], p[2 * mt][3], p[2 * mt + 1][3], xq.z, xq.w);
           }
         } else {
-          const float f0 = ue8m0_to_f32(lds8(sc_r0 + j)), f1 = ue8m0_to_f32(lds8(sc_r1 + j));
+          float f[4];
 #pragma unroll
-          for (int tl = 0; tl < 2; ++tl) {
-            if (tl < ntiles) {
-              const uint4 xq = lds128(xbase + tl * 8 * L.x_row + j * 64);
-              float part[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_16816(part, p0[0], p1[0], p0[1], p1[1], xq.x, xq.y);
-              mma_16816(part, p0[2], p1[2], p0[3], p1[3], xq.z, xq.w);
-              acc[tl][0] = fmaf(f0, part[0], acc[tl][0]);
-              acc[tl][1] = fmaf(f0, part[1], acc[tl][1]);
-              acc[tl][2] = fmaf(f1, part[2], acc[tl][2]);
-              acc[tl][3] = fmaf(f1, part[3], acc[tl][3]);
-            }
+          for (int m = 0; m < 4; ++m) f[m] = ldsf(lut + 4 * ((sb[m][0] >> (8 * jj)) & 0xFFu));
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            float part[4];
+            mma_16816_z(part, p[2 * mt][0], p[2 * mt + 1][0], p[2 * mt][1], p[2 * mt + 1][1], xq.x, xq.y);
+            mma_16816(part, p[2 * mt][2], p[2 * mt + 1][2], p[2 * mt][3], p[2 * mt + 1][3], xq.z, xq.w);
+            acc[mt][0] = fmaf(f[2 * mt], part[0], acc[mt][0]);
+            acc[mt][1] = fmaf(f[2 * mt], part[1], acc[mt][1]);
+            acc[mt][2] = fmaf(f[2 * mt + 1], part[2], acc[mt][2]);
+            acc[mt][3] = fmaf(f[2 * mt + 1], part[3], acc[mt][3]);
           }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
-    // ---- K halves meet in shared memory ----
-    named_bar_sync();
-    if (kh == 1) {
+    // ---- the four K quarters meet in shared memory, in a fixed order ----
+    float* bufA = red;
+    float* bufB = red + kRows * kRedPitch;
+    auto put = [&](float* b) {
 #pragma unroll
-      for (int tl = 0; tl < 2; ++tl) {
-        const int n = tl * 8 + 2 * t;
-        outs[r0 * kOutPitch + n] = acc[tl][0];
-        outs[r0 * kOutPitch + n + 1] = acc[tl][1];
-        outs[r1 * kOutPitch + n] = acc[tl][2];
-        outs[r1 * kOutPitch + n + 1] = acc[tl][3];
+      for (int mt = 0; mt < 2; ++mt) {
+        const int r = rbase + 16 * mt;
+        b[r * kRedPitch + 2 * t] = acc[mt][0];
+        b[r * kRedPitch + 2 * t + 1] = acc[mt][1];
+        b[(r + 8) * kRedPitch + 2 * t] = acc[mt][2];
+        b[(r + 8) * kRedPitch + 2 * t + 1] = acc[mt][3];
       }
+    };
+    auto add = [&](const float* b) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int r = rbase + 16 * mt;
+        acc[mt][0] += b[r * kRedPitch + 2 * t];
+        acc[mt][1] += b[r * kRedPitch + 2 * t + 1];
+        acc[mt][2] += b[(r + 8) * kRedPitch + 2 * t];
+        acc[mt][3] += b[(r + 8) * kRedPitch + 2 * t + 1];
+      }
+    };
+    named_bar_sync();                       // previous epilogue done with the buffers
+    if (kq == 2) put(bufA);
+    if (kq == 3) put(bufB);
+    named_bar_sync();
+    if (kq == 0) add(bufA);
+    if (kq == 1) add(bufB);
+    named_bar_sync();
+    if (kq == 1) put(bufA);
+    named_bar_sync();
+    if (kq == 0) {
+      add(bufA);
+      put(bufB);
     }
     named_bar_sync();
-    if (kh == 0) {
-#pragma unroll
-      for (int tl = 0; tl < 2; ++tl) {
-        const int n = tl * 8 + 2 * t;
-        outs[r0 * kOutPitch + n] += acc[tl][0];
-        outs[r0 * kOutPitch + n + 1] += acc[tl][1];
-        outs[r1 * kOutPitch + n] += acc[tl][2];
-        outs[r1 * kOutPitch + n + 1] += acc[tl][3];
-      }
-    }
-    named_bar_sync();
-    // ---- fused epilogue ----
+    // ---- fused epilogue (reads bufB) ----
     const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e] : 1.0f;
     if (kEpi == kEpiSwiglu) {
       for (int idx = threadIdx.x; idx < 32 * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 31, i = idx >> 5;
-        const int tok = a.perm[un.slot0 + i] / a.topk;
+        const int tok = perm_at(un.slot0 + i) / a.topk;
         const float sc = ldexpf(ts, a.sexp[tok]);
-        const float gv = fminf(outs[r * kOutPitch + i] * sc, a.limit);
-        const float uv = fminf(fmaxf(outs[(32 + r) * kOutPitch + i] * sc, -a.limit), a.limit);
+        const float gv = fminf(bufB[r * kRedPitch + i] * sc, a.limit);
+        const float uv = fminf(fmaxf(bufB[(32 + r) * kRedPitch + i] * sc, -a.limit), a.limit);
         const float hv = gv / (1.0f + expf(-gv)) * uv;
         a.h_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * 32 + r] = __float2half_rn(hv);
       }
     } else if (kEpi == kEpiDown) {
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
-        const float wgt = a.gw[a.perm[un.slot0 + i]];
+        const float wgt = a.gw[perm_at(un.slot0 + i)];
         a.o_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] =
-            outs[r * kOutPitch + i] * ts * wgt;
+            bufB[r * kRedPitch + i] * ts * wgt;
       }
     } else {
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
-        const float v = ldexpf(outs[r * kOutPitch + i] * ts, a.sexp[un.slot0 + i]);
+        const float v = ldexpf(bufB[r * kRedPitch + i] * ts, a.sexp[un.slot0 + i]);
         a.y_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] =
             __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
@@ -308,36 +490,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   finish();
 }
 
-Layout make_layout(int fmt, int K) {
+Layout make_layout(int fmt, int K, int E, int P) {
   Layout L{};
   const int B = (fmt == FP4_MXFP4) ? 32 : 16;
-  const int smem_cap = 227 * 1024 - 256;    // leave room for the kernel's static shared memory
-  const int extra = kRows * kOutPitch * 4 + 16 * kMaxStages + 1024;
-  for (int kc : {1024, 768, 512, 256}) {
-    if (K % kc != 0) continue;
-    Layout c{};
-    c.kc = kc;
-    c.nchunks = K / kc;
-    c.scale_row = kc / B;
-    c.codes_off = 0;
-    c.scales_off = kRows * kc / 2;
-    c.x_off = c.scales_off + kRows * c.scale_row;
-    c.x_row = 2 * kc + 64;
-    c.stage_bytes = static_cast<int>(align_up(c.x_off + kTok * c.x_row, 1024));
-    c.stages = std::min(kMaxStages, (smem_cap - extra) / c.stage_bytes);
-    if (c.stages < 2) continue;
-    c.out_off = c.stages * c.stage_bytes;
-    c.bar_off = c.out_off + kRows * kOutPitch * 4;
-    c.smem_bytes = c.bar_off + 16 * kMaxStages + 1024;   // + alignment slack
-    return c;
-  }
+  const int kc = (K % 512 == 0) ? 512 : ((K % 256 == 0) ? 256 : 0);
+  if (kc == 0) return L;
+  L.kc = kc;
+  L.nchunks = K / kc;
+  L.scale_row = kc / B;
+  L.codes_off = 0;
+  L.scales_off = kRows * kc / 2;
+  L.x_off = L.scales_off + kRows * L.scale_row;
+  L.x_row = 2 * kc + 64;
+  L.stage_bytes = static_cast<int>(align_up(L.x_off + kTok * L.x_row, 1024));
+  const int Eb = static_cast<int>(align_up(sizeof(int) * (E + 1), 16));
+  const int Cb = static_cast<int>(align_up(sizeof(int) * E, 16));
+  const int Pb = static_cast<int>(align_up(sizeof(int) * P, 16));
+  const int fixed = 2 * kRows * kRedPitch * 4 + 1024 + 3 * Eb + Cb + Pb + 16 * kMaxStages + 1024;
+  L.stages = std::min(kMaxStages, (kSmemBudget - fixed) / L.stage_bytes);
+  if (L.stages < 2 || L.stages * L.stage_bytes < static_cast<int>(sizeof(int)) * P) return Layout{};
+  L.red_off = L.stages * L.stage_bytes;
+  L.lut_off = L.red_off + 2 * kRows * kRedPitch * 4;
+  L.cnt_off = L.lut_off + 1024;
+  L.off_off = L.cnt_off + Eb;
+  L.pre_off = L.off_off + Eb;
+  L.perm_off = L.pre_off + Eb + Cb;
+  L.bar_off = L.perm_off + Pb;
+  L.smem_bytes = L.bar_off + 16 * kMaxStages + 1024;   // + alignment slack
   return L;
 }
 
-template <int kFmt, int kEpi>
-fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid,
-                      cudaStream_t st, bool pdl) {
-  auto kern = decode_kernel<kFmt, kEpi>;
+template <int kFmt, int kEpi, int kMode, int KC>
+fp4_status launch_kc(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
+                     bool pdl) {
+  auto kern = decode_kernel<kFmt, kEpi, kMode, KC>;
   static thread_local int configured = 0;
   if (configured < L.smem_bytes) {
     FP4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem_bytes));
@@ -346,28 +532,37 @@ fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& m
   return launch_pdl(kern, dim3(grid), dim3(kThreads), static_cast<size_t>(L.smem_bytes), st, pdl, map, a, L);
 }
 
+template <int kFmt, int kEpi, int kMode>
+fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
+                      bool pdl) {
+  if (L.kc == 512) return launch_kc<kFmt, kEpi, kMode, 512>(a, L, map, grid, st, pdl);
+  return launch_kc<kFmt, kEpi, kMode, 256>(a, L, map, grid, st, pdl);
+}
+
+template <int kFmt>
+fp4_status dispatch(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
+                    bool pdl) {
+  if (a.epi == kEpiSwiglu && a.mode == kModeRoute)
+    return launch_one<kFmt, kEpiSwiglu, kModeRoute>(a, L, map, grid, st, pdl);
+  if (a.epi == kEpiSwiglu) return launch_one<kFmt, kEpiSwiglu, kModeList>(a, L, map, grid, st, pdl);
+  if (a.epi == kEpiDown) return launch_one<kFmt, kEpiDown, kModeList>(a, L, map, grid, st, pdl);
+  return launch_one<kFmt, kEpiLinear, kModeStatic>(a, L, map, grid, st, pdl);
+}
+
 }  // namespace
 
 fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
-  const Layout L = make_layout(a.fmt, a.K);
+  const int E = (a.mode == kModeStatic) ? 1 : a.E;
+  const int P = (a.mode == kModeRoute) ? a.T * a.topk : 0;
+  const Layout L = make_layout(a.fmt, a.K, E, P);
   if (L.kc == 0) return FP4_ERR_UNSUPPORTED;
   CUtensorMap map;
   FP4_TRY(make_tmap_2d_u8(&map, a.codes, static_cast<uint64_t>(a.K / 2), static_cast<uint64_t>(a.rows_total),
                           static_cast<uint64_t>(a.K / 2), 128, 32, CU_TENSOR_MAP_SWIZZLE_128B));
-  int grid = num_sms();
-  if (a.units == nullptr) {
-    const int n = a.static_tiles * ((a.static_T + kTok - 1) / kTok);
-    grid = std::min(grid, n);
-  }
-  const int key = (a.fmt == FP4_NVFP4 ? 3 : 0) + a.epi;
-  switch (key) {
-    case 0: return launch_one<FP4_MXFP4, kEpiSwiglu>(a, L, map, grid, st, pdl);
-    case 1: return launch_one<FP4_MXFP4, kEpiDown>(a, L, map, grid, st, pdl);
-    case 2: return launch_one<FP4_MXFP4, kEpiLinear>(a, L, map, grid, st, pdl);
-    case 3: return launch_one<FP4_NVFP4, kEpiSwiglu>(a, L, map, grid, st, pdl);
-    case 4: return launch_one<FP4_NVFP4, kEpiDown>(a, L, map, grid, st, pdl);
-    default: return launch_one<FP4_NVFP4, kEpiLinear>(a, L, map, grid, st, pdl);
-  }
+  int grid = 2 * num_sms();
+  if (a.mode == kModeStatic) grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok));
+  return (a.fmt == FP4_NVFP4) ? dispatch<FP4_NVFP4>(a, L, map, grid, st, pdl)
+                              : dispatch<FP4_MXFP4>(a, L, map, grid, st, pdl);
 }
 
 // y[t, n] = bf16( sum_{j = 0..k-1} o[inv[t k + j], n] ), fixed j order.

@@ -26,16 +26,6 @@ fp4_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
   return FP4_OK;
 }
 
-// Per-expert work units {expert, row tile, first slot, tokens} for the grouped kernels.
-struct WorkListSpec {
-  int4* units_a;     // gate_up units (or null)
-  int4* units_b;     // down units (or null)
-  int tiles_a;       // row tiles per expert, list a
-  int tiles_b;
-  int tok_group;     // tokens per unit
-  int* n_units;      // [2] unit counts written by the router tail
-};
-
 struct RouteArgs {
   const void* x;
   const float* router_w;
@@ -52,7 +42,7 @@ struct RouteArgs {
   __half* x16;       // optional f16 copy of x with per-token power-of-two scale
   int* sexp;         // [T] the exponents
   WsControl* ctrl;   // workspace control block, reset by the first kernel (or null)
-  WorkListSpec wl;
+  bool logits_only;  // stop after R1 (the grouped kernel finishes routing itself)
   bool pdl_first;
 };
 
@@ -64,10 +54,18 @@ __global__ void x_to_f16_kernel(const uint16_t* __restrict__ x, int T, int H, __
 
 // Grouped decode GEMV (register dequantisation + warp-level MMA), see decode.cu.
 enum DecodeEpi { kEpiSwiglu = 0, kEpiDown = 1, kEpiLinear = 2 };
+// Where a grouped kernel finds its work units:
+//   kModeList:   counts / offsets / perm already in global memory;
+//   kModeRoute:  finish routing in the prologue from the logits (top-k, counts, perm);
+//   kModeStatic: dense layer, units follow from (N, T).
+enum DecodeMode { kModeList = 0, kModeRoute = 1, kModeStatic = 2 };
+constexpr int kRouteMaxPairs = 1024;   // kModeRoute limits (shared-memory routing state)
+constexpr int kRouteMaxExperts = 512;
 
 struct DecodeArgs {
   int fmt;                       // FP4_MXFP4 / FP4_NVFP4
   int epi;                       // DecodeEpi
+  int mode;                      // DecodeMode
   const uint8_t* codes;          // [rows_total, K/2]
   const uint8_t* scales;         // [rows_total, K/B]
   const float* tscale;           // [E] (NVFP4) or null
@@ -75,19 +73,18 @@ struct DecodeArgs {
   int K;
   int rows_per_expert;           // 2I (swiglu) or H (down) or N (linear)
   int inter;                     // I (swiglu: up rows start at I)
-  // units: device list (+ count) or the static linear mapping
-  const int4* units;
-  const int* n_units;
+  int E, T, topk;
+  const float* logits;           // kModeRoute: [T, E]
+  int32_t* ids;                  // kModeRoute: written by CTA 0
+  float* gw;                     // gate weights per pair (written by CTA 0 in kModeRoute)
+  int32_t* counts;               // [E]
+  int32_t* offsets;              // [E + 1]
+  int32_t* perm;                 // [P] slot -> pair
+  int32_t* inv;                  // [P] pair -> slot (written by CTA 0 in kModeRoute)
   int static_tiles;              // linear: N / 64
-  int static_T;                  // linear: T
-  // activations: f16 rows
-  const __half* x16;             // [rows, K]
+  const __half* x16;             // activation rows, f16 [rows, K]
   const int* sexp;               // per token exponent (swiglu / linear) or null
-  const int32_t* perm;           // swiglu/down: slot -> pair
-  int topk;
-  const float* gw;               // down: gate weights per pair
   float limit;                   // swiglu clamp
-  // outputs
   __half* h_out;                 // swiglu: [P, I]
   float* o_out;                  // down: [P, H]
   uint16_t* y_out;               // linear: [T, N] bf16

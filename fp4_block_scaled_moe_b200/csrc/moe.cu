@@ -12,23 +12,14 @@ namespace fp4 {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kTokGroupDecode = 16;
 
 struct MoeWs {
-  size_t status, n_units, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, units_a, units_b, h, o,
-      total;
-  int tiles_a, tiles_b;
-  int64_t max_units_a, max_units_b;
+  size_t status, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, h, o, total;
 };
 
 bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   const int64_t E = w->num_experts, H = w->hidden, I = w->inter;
   const int64_t P = static_cast<int64_t>(T) * k;
-  L->tiles_a = static_cast<int>(I / 32);
-  L->tiles_b = static_cast<int>(H / 64);
-  const int64_t groups = (P + kTokGroupDecode - 1) / kTokGroupDecode + std::min<int64_t>(E, P);
-  L->max_units_a = groups * L->tiles_a;
-  L->max_units_b = groups * L->tiles_b;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -36,7 +27,6 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
     return at;
   };
   L->status = take(sizeof(WsControl));
-  L->n_units = take(64);
   L->logits = take(sizeof(float) * T * E);
   L->ids = take(sizeof(int32_t) * P);
   L->gw = take(sizeof(float) * P);
@@ -46,8 +36,6 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   L->inv = take(sizeof(int32_t) * P);
   L->sexp = take(sizeof(int32_t) * T);
   L->x16 = take(sizeof(uint16_t) * T * H);
-  L->units_a = take(sizeof(int4) * L->max_units_a);
-  L->units_b = take(sizeof(int4) * L->max_units_b);
   L->h = take(sizeof(uint16_t) * P * I);
   L->o = take(sizeof(float) * P * H);
   L->total = off;
@@ -127,18 +115,16 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   ra.x16 = reinterpret_cast<__half*>(ws + L.x16);
   ra.sexp = reinterpret_cast<int*>(ws + L.sexp);
   ra.ctrl = reinterpret_cast<WsControl*>(ws + L.status);
-  ra.wl.units_a = reinterpret_cast<int4*>(ws + L.units_a);
-  ra.wl.units_b = reinterpret_cast<int4*>(ws + L.units_b);
-  ra.wl.tiles_a = L.tiles_a;
-  ra.wl.tiles_b = L.tiles_b;
-  ra.wl.tok_group = kTokGroupDecode;
-  ra.wl.n_units = reinterpret_cast<int*>(ws + L.n_units);
+  // small routing problems finish inside the gate_up kernel's prologue
+  const bool fused = P <= kRouteMaxPairs && E <= kRouteMaxExperts;
+  ra.logits_only = fused;
   ra.pdl_first = true;
   FP4_TRY(launch_route(ra, st));
 
   DecodeArgs g{};
   g.fmt = w->fmt;
   g.epi = kEpiSwiglu;
+  g.mode = fused ? kModeRoute : kModeList;
   g.codes = w->gu_codes;
   g.scales = w->gu_scales;
   g.tscale = w->gu_tscale;
@@ -146,13 +132,18 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   g.K = H;
   g.rows_per_expert = 2 * I;
   g.inter = I;
-  g.units = ra.wl.units_a;
-  g.n_units = ra.wl.n_units;
+  g.E = E;
+  g.T = T;
+  g.topk = k;
+  g.logits = ra.logits;
+  g.ids = ra.ids;
+  g.gw = ra.gw;
+  g.counts = ra.counts;
+  g.offsets = ra.offsets;
+  g.perm = ra.perm;
+  g.inv = ra.inv;
   g.x16 = ra.x16;
   g.sexp = ra.sexp;
-  g.perm = ra.perm;
-  g.topk = k;
-  g.gw = ra.gw;
   g.limit = w->swiglu_limit;
   g.h_out = reinterpret_cast<__half*>(ws + L.h);
   g.ldo = I;
@@ -162,14 +153,13 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
 
   DecodeArgs d = g;
   d.epi = kEpiDown;
+  d.mode = kModeList;
   d.codes = w->dn_codes;
   d.scales = w->dn_scales;
   d.tscale = w->dn_tscale;
   d.rows_total = static_cast<int64_t>(E) * H;
   d.K = I;
   d.rows_per_expert = H;
-  d.units = ra.wl.units_b;
-  d.n_units = ra.wl.n_units + 1;
   d.x16 = g.h_out;
   d.sexp = nullptr;
   d.o_out = reinterpret_cast<float*>(ws + L.o);
@@ -219,6 +209,8 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   DecodeArgs a{};
   a.fmt = fmt;
   a.epi = kEpiLinear;
+  a.mode = kModeStatic;
+  a.T = T;
   a.codes = codes;
   a.scales = scales;
   a.tscale = tensor_scale;
@@ -226,7 +218,6 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   a.K = static_cast<int>(K);
   a.rows_per_expert = static_cast<int>(N);
   a.static_tiles = static_cast<int>(N / 64);
-  a.static_T = T;
   a.x16 = x16;
   a.sexp = sexp;
   a.y_out = static_cast<uint16_t*>(y_bf16);

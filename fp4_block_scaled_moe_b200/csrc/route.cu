@@ -7,6 +7,7 @@
 #include <algorithm>
 
 #include "kernels.cuh"
+#include "routing.cuh"
 
 namespace fp4 {
 
@@ -60,11 +61,9 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
 
 // ---------------------------------------------------------------------------------
 // R1: logits[t, e] = sum_h x[t, h] w_r[e, h] + bias[e], float32 accumulation.
-// CTA = 8 warps = kExpPerCta experts x (8 / kExpPerCta) warps splitting H, for a group
-// of up to 16 tokens.  CTAs with blockIdx.x == 0 also convert their token rows to f16.
+// CTA (e, token group of 16): 8 warps split H; lanes stride by 4 floats.  The CTAs of
+// each token group also convert that group's rows of x to f16 (row i by CTA e = i mod E).
 // ---------------------------------------------------------------------------------
-constexpr int kExpPerCta = 2;
-constexpr int kWarpsPerExp = 8 / kExpPerCta;
 constexpr int kTokGroup = 16;
 
 __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict__ x,
@@ -81,33 +80,30 @@ __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict_
     s->done = 0u;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x;
   const int t0 = blockIdx.y * kTokGroup;
   const int nt = min(kTokGroup, T - t0);
-  if (x16 != nullptr && blockIdx.x == 0) {
-    for (int r = warp; r < nt; r += 8)
-      x_row_to_f16(x + static_cast<int64_t>(t0 + r) * H, H, x16 + static_cast<int64_t>(t0 + r) * H,
-                   sexp + t0 + r);
+  if (x16 != nullptr) {
+    for (int i = warp * E + e; i < nt; i += 8 * E)   // rows i with i % E == e, one warp each
+      x_row_to_f16(x + static_cast<int64_t>(t0 + i) * H, H, x16 + static_cast<int64_t>(t0 + i) * H,
+                   sexp + t0 + i);
   }
-  const int e = blockIdx.x * kExpPerCta + warp / kWarpsPerExp;
-  const int part = warp % kWarpsPerExp;
   float acc[kTokGroup];
 #pragma unroll
   for (int i = 0; i < kTokGroup; ++i) acc[i] = 0.f;
-  if (e < E) {
-    const int hspan = (H / kWarpsPerExp + 7) & ~7;
-    const int h0 = part * hspan, h1 = min(H, h0 + hspan);
-    const float* wrow = wr + static_cast<int64_t>(e) * H;
-    for (int h = h0 + lane * 4; h < h1; h += 128) {
-      const float4 wv = *reinterpret_cast<const float4*>(wrow + h);
+  const int hspan = ((H + 7) / 8 + 3) & ~3;
+  const int h0 = warp * hspan, h1 = min(H, h0 + hspan);
+  const float* wrow = wr + static_cast<int64_t>(e) * H;
+  for (int h = h0 + lane * 4; h < h1; h += 128) {
+    const float4 wv = *reinterpret_cast<const float4*>(wrow + h);
 #pragma unroll
-      for (int i = 0; i < kTokGroup; ++i) {
-        if (i < nt) {
-          const uint2 u = *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t0 + i) * H + h);
-          acc[i] = fmaf(__uint_as_float(u.x << 16), wv.x, acc[i]);
-          acc[i] = fmaf(__uint_as_float(u.x & 0xFFFF0000u), wv.y, acc[i]);
-          acc[i] = fmaf(__uint_as_float(u.y << 16), wv.z, acc[i]);
-          acc[i] = fmaf(__uint_as_float(u.y & 0xFFFF0000u), wv.w, acc[i]);
-        }
+    for (int i = 0; i < kTokGroup; ++i) {
+      if (i < nt) {
+        const uint2 u = *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t0 + i) * H + h);
+        acc[i] = fmaf(__uint_as_float(u.x << 16), wv.x, acc[i]);
+        acc[i] = fmaf(__uint_as_float(u.x & 0xFFFF0000u), wv.y, acc[i]);
+        acc[i] = fmaf(__uint_as_float(u.y << 16), wv.z, acc[i]);
+        acc[i] = fmaf(__uint_as_float(u.y & 0xFFFF0000u), wv.w, acc[i]);
       }
     }
   }
@@ -120,15 +116,12 @@ __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict_
 #pragma unroll
     for (int i = 0; i < kTokGroup; ++i) part_sum[warp][i] = acc[i];
   __syncthreads();
-  if (threadIdx.x < kExpPerCta * kTokGroup) {
-    const int le = threadIdx.x / kTokGroup, i = threadIdx.x % kTokGroup;
-    const int ee = blockIdx.x * kExpPerCta + le;
-    if (ee < E && i < nt) {
-      float s = 0.f;
-      for (int p = 0; p < kWarpsPerExp; ++p) s += part_sum[le * kWarpsPerExp + p][i];
-      if (bias) s += bias[ee];
-      logits[static_cast<int64_t>(t0 + i) * E + ee] = s;
-    }
+  if (threadIdx.x < nt) {
+    const int i = threadIdx.x;
+    float s = 0.f;
+    for (int p = 0; p < 8; ++p) s += part_sum[p][i];
+    if (bias) s += bias[e];
+    logits[static_cast<int64_t>(t0 + i) * E + e] = s;
   }
   pdl_launch_dependents();
 }
@@ -137,66 +130,13 @@ __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict_
 // R2: top-k per token (one warp per token) and softmax over the selected logits.
 // Order key: larger logit first; equal logits -> lower expert; NaN below every number.
 // ---------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t order_key(float v) {
-  if (v != v) return 0u;
-  v = v + 0.0f;                                    // -0 -> +0
-  const uint32_t b = __float_as_uint(v);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-constexpr int kMaxE = 1024;
-
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int32_t* __restrict__ ids, float* __restrict__ gw) {
   pdl_wait();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t < T) {
-    const float* lg = logits + static_cast<int64_t>(t) * E;
-    uint32_t key[kMaxE / 32];
-    const int per = (E + 31) / 32;
-#pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j) {
-      const int e = j * 32 + lane;
-      key[j] = (j < per && e < E) ? order_key(lg[e]) : 0u;
-    }
-    uint32_t taken = 0;   // bit j: my entry j already selected (or absent)
-#pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j)
-      if (!(j < per && j * 32 + lane < E)) taken |= 1u << j;
-    float sel_logit[32];
-    int sel_id[32];
-    for (int r = 0; r < k; ++r) {
-      uint32_t best = 0;
-      int best_e = 0x7FFFFFFF;
-#pragma unroll
-      for (int j = 0; j < kMaxE / 32; ++j) {
-        if (!(taken >> j & 1u)) {
-          const int e = j * 32 + lane;
-          if (key[j] > best || (key[j] == best && e < best_e)) { best = key[j]; best_e = e; }
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-        const int oe = __shfl_xor_sync(0xFFFFFFFFu, best_e, o);
-        if (ob > best || (ob == best && oe < best_e)) { best = ob; best_e = oe; }
-      }
-      if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
-      sel_id[r] = best_e;
-      sel_logit[r] = lg[best_e];
-    }
-    if (lane == 0) {
-      const float m = sel_logit[0];
-      float z[32];
-      float sum = 0.f;
-      for (int r = 0; r < k; ++r) { z[r] = expf(sel_logit[r] - m); sum += z[r]; }
-      for (int r = 0; r < k; ++r) {
-        ids[static_cast<int64_t>(t) * k + r] = sel_id[r];
-        gw[static_cast<int64_t>(t) * k + r] = z[r] / sum;
-      }
-    }
-  }
+  if (t < T)
+    topk_warp(logits + static_cast<int64_t>(t) * E, E, k, ids + static_cast<int64_t>(t) * k,
+              gw + static_cast<int64_t>(t) * k);
   pdl_launch_dependents();
 }
 
@@ -208,8 +148,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) perm_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                    int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                                    WorkListSpec wl) {
+                                                    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   extern __shared__ int32_t sm[];
   int32_t* hist = sm;                       // [32][E]
   int32_t* off = hist + 32 * E;             // [E + 1]
@@ -270,35 +209,6 @@ __global__ void __launch_bounds__(1024) perm_kernel(const int32_t* __restrict__ 
       inv[p] = slot;
     }
   }
-  // work lists: units {e, tile, slot0, ntok} ordered by expert, token group, tile
-  if (wl.units_a != nullptr) {
-    __syncthreads();
-    for (int list = 0; list < 2; ++list) {
-      int4* units = list == 0 ? wl.units_a : wl.units_b;
-      const int tiles = list == 0 ? wl.tiles_a : wl.tiles_b;
-      if (units == nullptr) continue;
-      const int e = threadIdx.x;
-      const int n = (e < E) ? (off[e + 1] - off[e]) : 0;
-      const int groups = (n + wl.tok_group - 1) / wl.tok_group;
-      const int cnt = groups * tiles;
-      scan[threadIdx.x] = cnt;
-      __syncthreads();
-      for (int o = 1; o < 1024; o <<= 1) {
-        const int add = (static_cast<int>(threadIdx.x) >= o) ? scan[threadIdx.x - o] : 0;
-        __syncthreads();
-        scan[threadIdx.x] += add;
-        __syncthreads();
-      }
-      int u = scan[threadIdx.x] - cnt;
-      if (threadIdx.x == 1023) wl.n_units[list] = scan[1023];
-      for (int g = 0; g < groups; ++g) {
-        const int s0 = off[e] + g * wl.tok_group;
-        const int nt = min(wl.tok_group, n - g * wl.tok_group);
-        for (int tl = 0; tl < tiles; ++tl) units[u++] = make_int4(e, tl, s0, nt);
-      }
-      __syncthreads();
-    }
-  }
   pdl_launch_dependents();
 }
 
@@ -307,7 +217,7 @@ size_t perm_smem_bytes(int E) { return (32 * static_cast<size_t>(E) + E + 1 + 10
 fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
   const int P = a.T * a.k;
   if (a.logits_in == nullptr) {
-    dim3 grid((a.E + kExpPerCta - 1) / kExpPerCta, (a.T + kTokGroup - 1) / kTokGroup);
+    dim3 grid(a.E, (a.T + kTokGroup - 1) / kTokGroup);
     FP4_TRY(launch_pdl(logits_kernel, grid, dim3(256), 0, st, a.pdl_first,
                        static_cast<const uint16_t*>(a.x), a.router_w, a.router_bias, a.T, a.H, a.E,
                        a.logits, a.x16, a.sexp, a.ctrl));
@@ -315,6 +225,7 @@ fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
     FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((a.T + 7) / 8), dim3(256), 0, st, a.pdl_first,
                        static_cast<const uint16_t*>(a.x), a.T, a.H, a.x16, a.sexp));
   }
+  if (a.logits_only) return FP4_OK;
   const float* lg = a.logits_in ? a.logits_in : a.logits;
   FP4_TRY(launch_pdl(topk_kernel, dim3((a.T + 7) / 8), dim3(256), 0, st, true, lg, a.T, a.E, a.k,
                      a.ids, a.gw));
@@ -326,7 +237,7 @@ fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
     configured_e = kMaxE;
   }
   FP4_TRY(launch_pdl(perm_kernel, dim3(1), dim3(1024), smem, st, true, a.ids, P, a.E, a.counts,
-                     a.offsets, a.perm, a.inv, a.wl));
+                     a.offsets, a.perm, a.inv));
   return FP4_OK;
 }
 
