@@ -12,6 +12,7 @@ from .api import (  # noqa: F401
     fp4_workspace_kernel_stats,
     fp4_workspace_status,
     moe_fp4_forward,
+    moe_fp4_forward_noalloc,
     moe_fp4_workspace_size,
     moe_route,
 )

@@ -60,6 +60,8 @@ SIGNATURES = {
     "fp4_linear_workspace_size": (_sz, [_i32, _i64]),
     "fp4_linear": (_cint, [_cint, _vp, _i32, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "fp4_workspace_status": (_cint, [_vp, _vp]),
+    "moe_fp4_noalloc_capacity": (_sz, []),
+    "moe_fp4_forward_noalloc": (_cint, [ctypes.POINTER(MoEWeightsC), _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "fp4_workspace_kernel_stats": (_cint, [_vp, _cint, ctypes.POINTER(KernelStatsC), _vp]),
 }
 

@@ -205,3 +205,18 @@ def fp4_workspace_kernel_stats(workspace, reset=False) -> dict:
         _ptr(workspace), 1 if reset else 0, ctypes.byref(st), _stream(workspace.device)))
     return {"gate_up_ns": st.gate_up_ns, "gate_up_launches": st.gate_up_launches,
             "down_ns": st.down_ns, "down_launches": st.down_launches}
+
+
+def moe_fp4_forward_noalloc(weights: MoEWeights, x, router_w, router_bias, k, y=None):
+    """The MoE layer without a caller workspace: scratch comes from the library's fixed
+    device buffer (see moe_fp4_forward_noalloc in include/fp4moe.h)."""
+    lib = L.load()
+    _need(x, "x", torch.bfloat16)
+    _need(router_w, "router_w", torch.float32)
+    T = x.shape[0]
+    s = weights.c_struct()
+    if y is None:
+        y = torch.empty((T, weights.H), dtype=torch.bfloat16, device=x.device)
+    L.check("moe_fp4_forward_noalloc", lib.moe_fp4_forward_noalloc(
+        ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(router_bias), T, k, _ptr(y), _stream(x.device)))
+    return y

@@ -206,6 +206,30 @@ fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K, 
 fp4_status fp4_workspace_status(const void* workspace, void* stream);
 
 /*
+ * moe_fp4_forward_noalloc: the same layer as moe_fp4_forward, for callers that cannot
+ * allocate device memory (no counterpart in the pages: an addition of this library).
+ * Some callers have no way to provide a workspace: a CUDA graph captured once that must
+ * not allocate again, a plugin whose host framework owns every allocation, or a
+ * real-time loop where an allocator call could block.  This entry point takes its
+ * scratch from a fixed buffer inside the library's own device memory instead, so the
+ * caller passes only inputs and outputs; it calls no cudaMalloc, no cudaFree and no
+ * allocating library routine.
+ *   - Capacity: moe_fp4_noalloc_capacity() bytes (16 MiB) on every device that loads the
+ *     library, held until the process exits.  A call whose moe_fp4_workspace_size(w, T, k)
+ *     exceeds it returns FP4_ERR_WORKSPACE and launches nothing (16 MiB covers decode
+ *     batches such as 64 tokens x top-8 at hidden 6144, intermediate 2048).
+ *   - The first call on a device looks up the buffer's device address and clears its
+ *     control block; make that first call before any stream capture on that device.
+ *   - All calls on a device share the one buffer and it keeps the previous call's
+ *     contents (each call rewrites everything it reads).  Calls that overlap on the GPU
+ *     -- on two streams, or from two host threads -- race on it: serialise them.
+ *   - Arguments, accuracy and errors otherwise as moe_fp4_forward (no routing outputs).
+ */
+size_t moe_fp4_noalloc_capacity(void);
+fp4_status moe_fp4_forward_noalloc(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
+                                   const float* router_bias, int32_t T, int32_t k, void* y_bf16, void* stream);
+
+/*
  * Per-kernel device time of the grouped expert kernels, accumulated in the workspace
  * by the kernels themselves from the device's global nanosecond timer: for each launch,
  * (last CTA finished) - (first CTA past its dependency wait).  Counters accumulate over
