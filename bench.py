@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=C.MOE_C2.name, choices=sorted(C.FULL))
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed CPU oracle sample")
     return ap.parse_args()
 
 
@@ -179,8 +180,10 @@ def run_ours(args, cfg, rank, world):
         with torch.cuda.stream(stream):
             step(c)                       # warm the launch path for this copy
             torch.cuda.synchronize()
+            n0 = api.fp4_launch_count()
             with torch.cuda.graph(g, stream=stream):
                 step(c)
+            launches_per_step = api.fp4_launch_count() - n0
         graphs.append(g)
     torch.cuda.synchronize()
     for i in range(args.warmup):
@@ -246,7 +249,7 @@ def run_ours(args, cfg, rank, world):
     kern_ms = {"gate_up": gu_ms, "down": dn_ms, "launches": kern["gate_up_launches"]}
     return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, e2e_ms=e2e_ms / args.steps,
                 kern=kern, kern_ms=kern_ms, clocks=clocks, copies=copies, counts=counts, status=status,
-                h2d=T * cfg.H * 2, d2h=T * cfg.H * 2)
+                h2d=T * cfg.H * 2, d2h=T * cfg.H * 2, launches_per_step=launches_per_step)
 
 
 # ------------------------------------------------------------------------------------
@@ -291,6 +294,26 @@ def roofline(cfg, r, hbm_peak, peaks):
             "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if "hbm_gbs" in peaks else "fallback",
             "bytes_per_launch": int(alg), "ms_per_launch": ms, "down_ms_per_launch": r["kern_ms"]["down"],
             "timer": "device globaltimer per launch, accumulated in the workspace over the timed steps"}
+
+
+def cpu_baseline(cfg, budget_s=20.0):
+    """The float64 oracle timed on this host's cores on a bounded sample of the same
+    workload: the layer for the first tokens (all their routed experts), repeated until
+    about budget_s of CPU time; value in the metric's unit (algorithmic GB/s)."""
+    n_tok = min(cfg.T, 4)
+    run, sample_bytes = oracle_sample(cfg, n_tok)
+    run()                                            # warm (dequantise caches, BLAS threads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt > budget_s or reps >= 50:
+            break
+    per = dt / reps
+    return {"value": sample_bytes / per / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {n_tok} of {cfg.T} tokens with all their routed experts, float64 numpy, "
+                      f"{reps} repetitions in {dt:.1f} s", "ms_per_sample": per * 1e3}
 
 
 def blas_threads():
@@ -354,11 +377,13 @@ def main():
                    "bytes_per_step": int(r["bytes_step"]), "pct_of_hbm_peak": 100 * value / world / hbm_peak},
         "e2e": {"value": r["bytes_step"] * world / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": r["launches_per_step"] * args.steps,
         "roofline": roofline(cfg, r, hbm_peak, peaks),
         "clocks": r["clocks"],
         "device_status": r["status"],
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -6,6 +6,7 @@ this package only marshals torch tensors into it.
 from .api import (  # noqa: F401
     MoEWeights,
     alloc_workspace,
+    fp4_launch_count,
     fp4_linear,
     fp4_pack,
     fp4_unpack,

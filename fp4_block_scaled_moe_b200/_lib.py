@@ -51,6 +51,7 @@ SIGNATURES = {
     "fp4_status_string": (ctypes.c_char_p, [_cint]),
     "fp4_last_error_string": (ctypes.c_char_p, []),
     "fp4_version": (ctypes.c_char_p, []),
+    "fp4_launch_count": (ctypes.c_ulonglong, []),
     "fp4_pack": (_cint, [_cint, _vp, _cint, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "fp4_unpack": (_cint, [_cint, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _cint, _vp]),
     "moe_route": (_cint, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),

@@ -193,6 +193,11 @@ def fp4_linear(x, codes, scales, tensor_scale=None, fmt="mxfp4", workspace=None,
     return y
 
 
+def fp4_launch_count() -> int:
+    """Kernel launches the library has issued in this process (see include/fp4moe.h)."""
+    return int(L.load().fp4_launch_count())
+
+
 def fp4_workspace_status(workspace) -> str:
     code = L.load().fp4_workspace_status(_ptr(workspace), _stream(workspace.device))
     return L.STATUS.get(code, str(code))

@@ -1,3 +1,4 @@
+#include <atomic>
 // C-ABI plumbing: status strings, CUDA error capture, device queries, tensor maps,
 // and the workspace status word.
 #include <cudaTypedefs.h>
@@ -89,6 +90,13 @@ extern "C" const char* fp4_status_string(fp4_status s) {
 extern "C" const char* fp4_last_error_string(void) { return g_last_error; }
 
 extern "C" const char* fp4_version(void) { return "0.1.0"; }
+
+namespace fp4 {
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace fp4
+
+extern "C" unsigned long long fp4_launch_count(void) { return fp4::g_launches.load(std::memory_order_relaxed); }
 
 extern "C" fp4_status fp4_workspace_status(const void* workspace, void* stream) {
   if (workspace == nullptr) return FP4_ERR_INVALID_ARG;

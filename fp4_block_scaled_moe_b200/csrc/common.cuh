@@ -16,6 +16,8 @@ namespace fp4 {
 // ------------------------------------------------------------------------------------
 
 fp4_status record_cuda_error(cudaError_t e, const char* where);
+// Count one accepted kernel launch (process-wide; read by fp4_launch_count).
+void note_launch(unsigned n = 1);
 
 #define FP4_TRY_CUDA(call)                                         \
   do {                                                             \
@@ -73,7 +75,8 @@ struct KernelSlot {
 };
 struct WsControl {
   uint32_t status;
-  uint32_t pad[3];
+  uint32_t unit_next[2];          // dynamic work-unit counters of the grouped kernels (gate_up, down)
+  uint32_t pad;
   KernelSlot slot[2];             // 0: gate_up, 1: down
 };
 static_assert(sizeof(WsControl) <= 256, "control block");
@@ -216,7 +219,7 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
 // D = A (16x16 f16, row) * B (16x8 f16, col) + C, f32 accumulate.
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9},"
       " {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -227,7 +230,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 __device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                             uint32_t b0, uint32_t b1) {
   const float z = 0.0f;
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9},"
       " {%10, %10, %10, %10};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])

@@ -45,7 +45,8 @@ struct Layout {
   int x_row;         // bytes per token row in the stage (padded)
   int stage_bytes;
   int stages;
-  int red_off;       // 2 x [64][kRedPitch] fp32
+  int red_off;       // 4 x [64][kRedPitch] fp32 (one per K quarter)
+  int su_off;        // [kMaxStages] int: work unit of each ring stage
   int lut_off;       // 256 fp32 (UE8M0 -> float)
   int cnt_off, off_off, pre_off;   // [E + 1] int each (pre is followed by [E] cursors)
   int perm_off;      // [P] int (kModeRoute)
@@ -55,36 +56,6 @@ struct Layout {
 
 __device__ __forceinline__ void named_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float ldsf(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds16u(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds8(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
 }
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -277,12 +248,34 @@ __global__ void __launch_bounds__(kThreads, 2)
     return a.perm[slot];
   };
   constexpr int ncb = KC / 256;                                // 128-byte code boxes per row per stage
+  int* stage_unit = reinterpret_cast<int*>(smem + L.su_off);
+  // work units: the first is blockIdx.x, later ones come from a counter (zeroed by the router)
+  auto next_unit = [&](int u) -> int {
+    if (kMode == kModeStatic || a.unit_next == nullptr) return u + static_cast<int>(gridDim.x);
+    int v = 0;
+    if (lane == 0) v = static_cast<int>(gridDim.x + atomicAdd(a.unit_next, 1u));
+    return __shfl_sync(0xFFFFFFFFu, v, 0);
+  };
 
   if (warp == kConsumers) {
     // ------------------------------- producer -------------------------------------
     int it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    int u = blockIdx.x;
+    while (true) {
+      if (u >= n_units) {
+        // sentinel stage: no more work for this CTA
+        const int s = it % L.stages;
+        if (it >= L.stages &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / L.stages) & 1) ^ 1, a.status)))
+          break;
+        if (lane == 0) {
+          stage_unit[s] = -1;
+          mbar_arrive(bar_full + 8 * s);
+        }
+        ++it;
+        break;
+      }
       const Unit un = get_unit(u);
       const int64_t y0 = unit_row<kEpi>(a, un, 0), y1 = unit_row<kEpi>(a, un, 32);
       int xr = 0;
@@ -291,10 +284,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       constexpr int words = kScaleRow / 4;
       for (int c = 0; c < L.nchunks; ++c, ++it) {
         const int s = it % L.stages;
-        if (it >= L.stages && !mbar_wait(bar_empty + 8 * s, ((it / L.stages) & 1) ^ 1, a.status)) {
+        if (it >= L.stages &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / L.stages) & 1) ^ 1, a.status))) {
           ok = false;
           break;
         }
+        if (lane == 0) stage_unit[s] = u;
         const uint32_t st_base = sbase + s * L.stage_bytes;
         const int k0 = c * KC;
         for (int w = lane; w < kRows * words; w += 32) {
@@ -315,6 +310,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           bulk_g2s(st_base + kXOff + lane * kXRow, a.x16 + static_cast<int64_t>(xr) * a.K + k0,
                    static_cast<uint32_t>(KC * 2), bar_full + 8 * s);
       }
+      if (!ok) break;
+      u = next_unit(u);
     }
     // drain: never leave while copies into this CTA's shared memory are in flight
     for (int d = 1; d <= L.stages && d <= it; ++d) {
@@ -330,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int g = lane >> 2, t = lane & 3;
   const int rbase = 32 * rh + g;                 // rows rbase + 8m, m = 0..3
   float* red = reinterpret_cast<float*>(smem + L.red_off);
-  const uint32_t lut = sbase + L.lut_off;
+  const float* lut_f = reinterpret_cast<const float*>(smem + L.lut_off);
   const int jbase = kq * kNq;                    // this warp's first 32-K region of a stage
   // per-thread offsets within a stage: codes (swizzled 128-byte rows), scales, activations
   const uint32_t c_off = ((jbase >> 3) * kRows + rbase) * 128 + 4 * t;
@@ -340,7 +337,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t s_off = kScalesOff + rbase * kScaleRow + (kFmt == FP4_MXFP4 ? jbase : 2 * jbase);
   const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
   int it = 0;
-  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+  while (true) {
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * (it % L.stages), (it / L.stages) & 1, a.status))) {
+      finish();
+      return;
+    }
+    const int u = *reinterpret_cast<volatile int*>(&stage_unit[it % L.stages]);
+    if (u < 0) break;                              // sentinel: no more work
     const Unit un = get_unit(u);
     float acc[2][4];
 #pragma unroll
@@ -349,38 +352,39 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
     for (int c = 0; c < L.nchunks; ++c, ++it) {
       const int s = it % L.stages;
-      if (!mbar_wait(bar_full + 8 * s, (it / L.stages) & 1, a.status)) {
+      if (c > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s, (it / L.stages) & 1, a.status))) {
         finish();
         return;
       }
-      const uint32_t st_base = sbase + s * L.stage_bytes;
+      // plain shared-memory loads (ordered after the barrier wait, free to be scheduled)
+      const uint8_t* stp = smem + s * L.stage_bytes;
       // scale bytes of this warp's regions, one load per row
       uint32_t sb[4][(kFmt == FP4_MXFP4) ? 1 : 2];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const uint32_t addr = st_base + s_off + m * 8 * kScaleRow;
+        const uint8_t* sp = stp + s_off + m * 8 * kScaleRow;
         if (kFmt == FP4_MXFP4) {
           static_assert(kFmt != FP4_MXFP4 || kNq <= 4, "scale word");
-          sb[m][0] = (kNq == 4) ? lds32(addr) : lds16u(addr);
+          sb[m][0] = (kNq == 4) ? *reinterpret_cast<const uint32_t*>(sp) : *reinterpret_cast<const uint16_t*>(sp);
         } else if (kNq == 4) {
-          const uint2 v = lds64(addr);                 // 2 kNq = 8 bytes
+          const uint2 v = *reinterpret_cast<const uint2*>(sp);      // 2 kNq = 8 bytes
           sb[m][0] = v.x;
           sb[m][(kFmt == FP4_MXFP4) ? 0 : 1] = v.y;
         } else {
-          sb[m][0] = lds32(addr);                      // 2 kNq = 4 bytes
+          sb[m][0] = *reinterpret_cast<const uint32_t*>(sp);        // 2 kNq = 4 bytes
           sb[m][(kFmt == FP4_MXFP4) ? 0 : 1] = 0u;
         }
       }
 #pragma unroll
       for (int jj = 0; jj < kNq; ++jj) {
-        const uint32_t caddr = st_base + c_off + c_xo[jj];
+        const uint8_t* cp = stp + c_off + c_xo[jj];
         uint32_t w[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) w[m] = lds32(caddr + m * 8 * 128);
+        for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(cp + m * 8 * 128);
         uint32_t p[4][4];
 #pragma unroll
         for (int m = 0; m < 4; ++m) e2m1x8_to_f16x8(w[m], p[m][0], p[m][1], p[m][2], p[m][3]);
-        const uint4 xq = lds128(st_base + x_off + jj * 64);
+        const uint4 xq = *reinterpret_cast<const uint4*>(stp + x_off + jj * 64);
         if (kFmt == FP4_NVFP4) {
           // this thread's 8 K positions lie in block 2j + (t >> 1): byte 2 jj + (t >> 1) of the row's run
           const int bsel = 2 * jj + (t >> 1);
@@ -406,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         } else {
           float f[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) f[m] = ldsf(lut + 4 * ((sb[m][0] >> (8 * jj)) & 0xFFu));
+          for (int m = 0; m < 4; ++m) f[m] = lut_f[(sb[m][0] >> (8 * jj)) & 0xFFu];
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt) {
             float part[4];
@@ -422,10 +426,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
-    // ---- the four K quarters meet in shared memory, in a fixed order ----
-    float* bufA = red;
-    float* bufB = red + kRows * kRedPitch;
-    auto put = [&](float* b) {
+    // ---- the four K quarters meet in shared memory; summed in a fixed order ----
+    named_bar_sync();                       // the previous unit's epilogue is done with red
+    {
+      float* b = red + kq * kRows * kRedPitch;
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         const int r = rbase + 16 * mt;
@@ -434,40 +438,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         b[(r + 8) * kRedPitch + 2 * t] = acc[mt][2];
         b[(r + 8) * kRedPitch + 2 * t + 1] = acc[mt][3];
       }
-    };
-    auto add = [&](const float* b) {
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int r = rbase + 16 * mt;
-        acc[mt][0] += b[r * kRedPitch + 2 * t];
-        acc[mt][1] += b[r * kRedPitch + 2 * t + 1];
-        acc[mt][2] += b[(r + 8) * kRedPitch + 2 * t];
-        acc[mt][3] += b[(r + 8) * kRedPitch + 2 * t + 1];
-      }
-    };
-    named_bar_sync();                       // previous epilogue done with the buffers
-    if (kq == 2) put(bufA);
-    if (kq == 3) put(bufB);
-    named_bar_sync();
-    if (kq == 0) add(bufA);
-    if (kq == 1) add(bufB);
-    named_bar_sync();
-    if (kq == 1) put(bufA);
-    named_bar_sync();
-    if (kq == 0) {
-      add(bufA);
-      put(bufB);
     }
     named_bar_sync();
-    // ---- fused epilogue (reads bufB) ----
+    auto val = [&](int r, int i) {
+      const int o = r * kRedPitch + i, q = kRows * kRedPitch;
+      return ((red[o] + red[q + o]) + red[2 * q + o]) + red[3 * q + o];
+    };
+    // ---- fused epilogue ----
     const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e] : 1.0f;
     if (kEpi == kEpiSwiglu) {
       for (int idx = threadIdx.x; idx < 32 * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 31, i = idx >> 5;
         const int tok = perm_at(un.slot0 + i) / a.topk;
         const float sc = ldexpf(ts, a.sexp[tok]);
-        const float gv = fminf(bufB[r * kRedPitch + i] * sc, a.limit);
-        const float uv = fminf(fmaxf(bufB[(32 + r) * kRedPitch + i] * sc, -a.limit), a.limit);
+        const float gv = fminf(val(r, i) * sc, a.limit);
+        const float uv = fminf(fmaxf(val(32 + r, i) * sc, -a.limit), a.limit);
         const float hv = gv / (1.0f + expf(-gv)) * uv;
         a.h_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * 32 + r] = __float2half_rn(hv);
       }
@@ -475,13 +460,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
         const float wgt = a.gw[perm_at(un.slot0 + i)];
-        a.o_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] =
-            bufB[r * kRedPitch + i] * ts * wgt;
+        a.o_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] = val(r, i) * ts * wgt;
       }
     } else {
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
-        const float v = ldexpf(bufB[r * kRedPitch + i] * ts, a.sexp[un.slot0 + i]);
+        const float v = ldexpf(val(r, i) * ts, a.sexp[un.slot0 + i]);
         a.y_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] =
             __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
@@ -506,11 +490,12 @@ Layout make_layout(int fmt, int K, int E, int P) {
   const int Eb = static_cast<int>(align_up(sizeof(int) * (E + 1), 16));
   const int Cb = static_cast<int>(align_up(sizeof(int) * E, 16));
   const int Pb = static_cast<int>(align_up(sizeof(int) * P, 16));
-  const int fixed = 2 * kRows * kRedPitch * 4 + 1024 + 3 * Eb + Cb + Pb + 16 * kMaxStages + 1024;
+  const int fixed = 4 * kRows * kRedPitch * 4 + 4 * kMaxStages + 1024 + 3 * Eb + Cb + Pb + 16 * kMaxStages + 1024;
   L.stages = std::min(kMaxStages, (kSmemBudget - fixed) / L.stage_bytes);
   if (L.stages < 2 || L.stages * L.stage_bytes < static_cast<int>(sizeof(int)) * P) return Layout{};
   L.red_off = L.stages * L.stage_bytes;
-  L.lut_off = L.red_off + 2 * kRows * kRedPitch * 4;
+  L.su_off = L.red_off + 4 * kRows * kRedPitch * 4;
+  L.lut_off = L.su_off + 4 * kMaxStages;
   L.cnt_off = L.lut_off + 1024;
   L.off_off = L.cnt_off + Eb;
   L.pre_off = L.off_off + Eb;
@@ -565,7 +550,7 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
                               : dispatch<FP4_MXFP4>(a, L, map, grid, st, pdl);
 }
 
-// y[t, n] = bf16( sum_{j = 0..k-1} o[inv[t k + j], n] ), fixed j order.
+// y[t, n] = bf16( sum_{j = 0..k-1} o[inv[t k + j], n] ), fixed j order (deterministic).
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv,
                                                       int T, int k, int H, uint16_t* __restrict__ y) {
   pdl_wait();

@@ -23,6 +23,7 @@ fp4_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
   cfg.numAttrs = pdl ? 1 : 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e != cudaSuccess) return record_cuda_error(e, "cudaLaunchKernelEx");
+  note_launch();
   return FP4_OK;
 }
 
@@ -91,11 +92,14 @@ struct DecodeArgs {
   int ldo;                       // leading dim of the output rows
   uint32_t* status;
   KernelSlot* slot;              // per-launch device timing (or null)
+  uint32_t* unit_next;           // dynamic scheduling counter (zeroed by the router), or null
 };
 
 fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl);
 
-__global__ void combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv, int T, int k,
-                               int H, uint16_t* __restrict__ y);
+// y[t, :] = bf16(sum_j o[inv[t k + j], :]) in j order.
+__global__ void combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv, int T, int k, int H,
+                               uint16_t* __restrict__ y);
+
 
 }  // namespace fp4

@@ -149,6 +149,7 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   g.ldo = I;
   g.status = &ra.ctrl->status;
   g.slot = &ra.ctrl->slot[0];
+  g.unit_next = &ra.ctrl->unit_next[0];
   FP4_TRY(launch_decode(g, st, true));
 
   DecodeArgs d = g;
@@ -164,6 +165,7 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   d.sexp = nullptr;
   d.o_out = reinterpret_cast<float*>(ws + L.o);
   d.slot = &ra.ctrl->slot[1];
+  d.unit_next = &ra.ctrl->unit_next[1];
   d.ldo = H;
   FP4_TRY(launch_decode(d, st, true));
 
@@ -172,7 +174,6 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   FP4_TRY(launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, true,
                      static_cast<const float*>(d.o_out), static_cast<const int32_t*>(ra.inv), T, k, H,
                      static_cast<uint16_t*>(y_bf16)));
-  (void)P;
   return FP4_OK;
 }
 

@@ -284,6 +284,7 @@ extern "C" fp4_status fp4_pack(fp4_format fmt, const void* w, fp4_dtype w_dtype,
       mxfp4_pack_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
           static_cast<const __nv_bfloat16*>(w), n4, reinterpret_cast<uint16_t*>(codes), scales);
     FP4_TRY_CUDA(cudaGetLastError());
+    note_launch(1);
     return FP4_OK;
   }
   if (batch > 65535) return FP4_ERR_UNSUPPORTED;
@@ -305,6 +306,7 @@ extern "C" fp4_status fp4_pack(fp4_format fmt, const void* w, fp4_dtype w_dtype,
   }
   nvfp4_finalize_kernel<<<static_cast<unsigned>((batch + 255) / 256), 256, 0, st>>>(tensor_scale, batch);
   FP4_TRY_CUDA(cudaGetLastError());
+  note_launch(3);
   return FP4_OK;
 }
 
@@ -336,5 +338,6 @@ extern "C" fp4_status fp4_unpack(fp4_format fmt, const uint8_t* codes, const uin
       unpack_kernel<FP4_NVFP4, FP4_BF16><<<grid, kThreads, 0, st>>>(codes, scales, tensor_scale, per, total, out);
   }
   FP4_TRY_CUDA(cudaGetLastError());
+  note_launch(1);
   return FP4_OK;
 }

@@ -61,41 +61,91 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
 
 // ---------------------------------------------------------------------------------
 // R1: logits[t, e] = sum_h x[t, h] w_r[e, h] + bias[e], float32 accumulation.
-// CTA (e, token group of 16): 8 warps split H; lanes stride by 4 floats.  The CTAs of
-// each token group also convert that group's rows of x to f16 (row i by CTA e = i mod E).
+// CTA (e, token group of 16), 16 warps splitting H.  The router weights do not depend
+// on the previous kernel, so the first slice of them is fetched before the dependency
+// wait.  CTA (e, group) also converts row e (+ multiples of E) of the group to f16, and
+// CTA (0, 0) clears the per-call counters of the grouped kernels.
 // ---------------------------------------------------------------------------------
 constexpr int kTokGroup = 16;
+constexpr int kLogitsWarps = 16;
+constexpr int kWrPrefetch = 4;   // float4 per lane fetched before the dependency wait
 
-__global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict__ x,
-                                                     const float* __restrict__ wr,
-                                                     const float* __restrict__ bias, int T, int H, int E,
-                                                     float* __restrict__ logits, __half* __restrict__ x16,
-                                                     int* __restrict__ sexp, WsControl* __restrict__ ctrl) {
+// f16 copy of one row with the whole CTA: x16 = x * 2^-s, max|x| * 2^-s in [2^14, 2^15)
+__device__ void x_row_to_f16_cta(const uint16_t* __restrict__ xrow, int H, __half* __restrict__ out,
+                                 int* __restrict__ sexp, float* red) {
+  float amax = 0.f;
+  for (int h = threadIdx.x * 8; h < H; h += blockDim.x * 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xrow + h);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
+  __syncthreads();
+  int s = 0;
+  if (amax > 0.f && isfinite(amax)) {
+    int e;
+    frexpf(amax, &e);            // amax = f 2^e, f in [0.5, 1): floor(log2 amax) = e - 1
+    s = (e - 1) - 14;
+  }
+  for (int h = threadIdx.x * 8; h < H; h += blockDim.x * 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xrow + h);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half lo = __float2half_rn(ldexpf(__uint_as_float(w[j] << 16), -s));
+      const __half hi = __float2half_rn(ldexpf(__uint_as_float(w[j] & 0xFFFF0000u), -s));
+      o[j] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+    }
+    *reinterpret_cast<uint4*>(out + h) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (threadIdx.x == 0) *sexp = s;
+}
+
+__global__ void __launch_bounds__(kLogitsWarps * 32) logits_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias, int T, int H,
+    int E, float* __restrict__ logits, __half* __restrict__ x16, int* __restrict__ sexp,
+    WsControl* __restrict__ ctrl) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x;
+  const int hspan = ((H + kLogitsWarps - 1) / kLogitsWarps + 3) & ~3;
+  const int h0 = warp * hspan, h1 = min(H, h0 + hspan);
+  const float* wrow = wr + static_cast<int64_t>(e) * H;
+  float4 wpre[kWrPrefetch];
+#pragma unroll
+  for (int q = 0; q < kWrPrefetch; ++q) {
+    const int h = h0 + lane * 4 + q * 128;
+    wpre[q] = (h < h1) ? *reinterpret_cast<const float4*>(wrow + h) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   pdl_wait();
   if (ctrl != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) {
     if (threadIdx.x == 0) ctrl->status = 0u;
+    ctrl->unit_next[threadIdx.x] = 0u;
     KernelSlot* s = &ctrl->slot[threadIdx.x];
     s->start_min = ~0ull;
     s->end_max = 0ull;
     s->done = 0u;
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x;
+  __shared__ float red[kLogitsWarps];
   const int t0 = blockIdx.y * kTokGroup;
   const int nt = min(kTokGroup, T - t0);
-  if (x16 != nullptr) {
-    for (int i = warp * E + e; i < nt; i += 8 * E)   // rows i with i % E == e, one warp each
-      x_row_to_f16(x + static_cast<int64_t>(t0 + i) * H, H, x16 + static_cast<int64_t>(t0 + i) * H,
-                   sexp + t0 + i);
-  }
+  if (x16 != nullptr)
+    for (int i = e; i < nt; i += E)
+      x_row_to_f16_cta(x + static_cast<int64_t>(t0 + i) * H, H, x16 + static_cast<int64_t>(t0 + i) * H,
+                       sexp + t0 + i, red);
   float acc[kTokGroup];
 #pragma unroll
   for (int i = 0; i < kTokGroup; ++i) acc[i] = 0.f;
-  const int hspan = ((H + 7) / 8 + 3) & ~3;
-  const int h0 = warp * hspan, h1 = min(H, h0 + hspan);
-  const float* wrow = wr + static_cast<int64_t>(e) * H;
-  for (int h = h0 + lane * 4; h < h1; h += 128) {
-    const float4 wv = *reinterpret_cast<const float4*>(wrow + h);
+  auto accumulate = [&](const float4 wv, int h) {
 #pragma unroll
     for (int i = 0; i < kTokGroup; ++i) {
       if (i < nt) {
@@ -106,22 +156,29 @@ __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict_
         acc[i] = fmaf(__uint_as_float(u.y & 0xFFFF0000u), wv.w, acc[i]);
       }
     }
+  };
+#pragma unroll
+  for (int q = 0; q < kWrPrefetch; ++q) {
+    const int h = h0 + lane * 4 + q * 128;
+    if (h < h1) accumulate(wpre[q], h);
   }
+  for (int h = h0 + lane * 4 + kWrPrefetch * 128; h < h1; h += 128)
+    accumulate(*reinterpret_cast<const float4*>(wrow + h), h);
 #pragma unroll
   for (int i = 0; i < kTokGroup; ++i)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
-  __shared__ float part_sum[8][kTokGroup];
+  __shared__ float part_sum[kLogitsWarps][kTokGroup];
   if (lane == 0)
 #pragma unroll
     for (int i = 0; i < kTokGroup; ++i) part_sum[warp][i] = acc[i];
   __syncthreads();
   if (threadIdx.x < nt) {
     const int i = threadIdx.x;
-    float s = 0.f;
-    for (int p = 0; p < 8; ++p) s += part_sum[p][i];
-    if (bias) s += bias[e];
-    logits[static_cast<int64_t>(t0 + i) * E + e] = s;
+    float sum = 0.f;
+    for (int p = 0; p < kLogitsWarps; ++p) sum += part_sum[p][i];
+    if (bias) sum += bias[e];
+    logits[static_cast<int64_t>(t0 + i) * E + e] = sum;
   }
   pdl_launch_dependents();
 }
@@ -218,7 +275,7 @@ fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
   const int P = a.T * a.k;
   if (a.logits_in == nullptr) {
     dim3 grid(a.E, (a.T + kTokGroup - 1) / kTokGroup);
-    FP4_TRY(launch_pdl(logits_kernel, grid, dim3(256), 0, st, a.pdl_first,
+    FP4_TRY(launch_pdl(logits_kernel, grid, dim3(kLogitsWarps * 32), 0, st, a.pdl_first,
                        static_cast<const uint16_t*>(a.x), a.router_w, a.router_bias, a.T, a.H, a.E,
                        a.logits, a.x16, a.sexp, a.ctrl));
   } else if (a.x16 != nullptr) {

@@ -69,6 +69,10 @@ const char* fp4_status_string(fp4_status s);
 const char* fp4_last_error_string(void);
 /* Library version, e.g. "0.1.0". */
 const char* fp4_version(void);
+/* Number of CUDA kernel launches this library has issued in this process so far (all
+ * entry points, all devices and streams; counted on the host when a launch is accepted,
+ * whether it later runs or is captured into a graph).  Never fails. */
+unsigned long long fp4_launch_count(void);
 
 /*
  * fp4_pack: quantise `batch` matrices w [batch, n, k] (float32 or bf16, device) to
