@@ -34,6 +34,7 @@ class MoEWeightsC(ctypes.Structure):
         ("dn_codes", _vp), ("dn_scales", _vp), ("dn_tscale", _vp),
         ("gu_cb", _vp), ("gu_rowptr", _vp), ("gu_col", _vp), ("gu_val", _vp),
         ("dn_cb", _vp), ("dn_rowptr", _vp), ("dn_col", _vp), ("dn_val", _vp),
+        ("kernel_variant", _i32),
     ]
 
 

@@ -127,12 +127,15 @@ class MoEWeights:
     dn_rowptr: torch.Tensor | None = None
     dn_col: torch.Tensor | None = None
     dn_val: torch.Tensor | None = None
+    # expert-GEMM kernels: 0 chosen per call, 1 CUDA-core GEMV, 2 tensor-core (MXFP4)
+    kernel_variant: int = 0
 
     def c_struct(self):
         s = L.MoEWeightsC()
         s.fmt = fmt_code(self.fmt)
         s.num_experts, s.hidden, s.inter = self.E, self.H, self.I
         s.swiglu_limit = self.swiglu_limit
+        s.kernel_variant = self.kernel_variant
         for name in ("gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales", "dn_tscale", "gu_cb",
                      "gu_rowptr", "gu_col", "gu_val", "dn_cb", "dn_rowptr", "dn_col", "dn_val"):
             t = getattr(self, name)

@@ -46,26 +46,32 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-fp4_status make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows,
-                           uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
-                           CUtensorMapSwizzle swz) {
+fp4_status make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner_elems,
+                        uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                        CUtensorMapSwizzle swz) {
   auto enc = get_encode();
   if (enc == nullptr) {
     std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
     return FP4_ERR_CUDA;
   }
-  cuuint64_t dims[2] = {inner_bytes, rows};
+  cuuint64_t dims[2] = {inner_elems, rows};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
     return FP4_ERR_CUDA;
   }
   return FP4_OK;
+}
+
+fp4_status make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows,
+                           uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                           CUtensorMapSwizzle swz) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner_bytes, rows, row_stride_bytes, box_inner,
+                      box_rows, swz);
 }
 
 }  // namespace fp4

@@ -1,0 +1,538 @@
+// Grouped MXFP4 expert GEMMs on the block-scaled tensor cores (tcgen05.mma
+// kind::mxf8f6f4): the 4-bit weights go from HBM to shared memory by TMA and straight
+// into the MMA with their UE8M0 block scales; no CUDA core touches a weight.
+//
+// Format: MXFP4 as "XFP：质量地板驱动的自适应码本量化" (section 路线二) describes it, E2M1
+// elements with one power-of-two scale per 32.  The bf16 activations keep their accuracy
+// by entering the MMA as the sum of two MXFP8 terms (E4M3 elements, UE8M0 scale per 32):
+// x = t1 + t2 with t1 = E4M3(x / s1) s1 and t2 = E4M3((x - t1) / s2) s2, leaving about
+// 2^-8 |x| per element.  The two terms of token slot i are B rows 2i and 2i + 1, so the
+// product with x_i is D[:, 2i] + D[:, 2i + 1].
+//
+// Warp roles of one persistent CTA per SM:
+//   warp 0     producer: TMA of the weight tile (FP4 widened to 16-byte slots, 128-byte
+//              swizzle) and of the activation-term tile; 4-byte async copies place the
+//              scale bytes in the 32-row x 16-byte atoms the TMEM scale copy reads.
+//   warp 1     MMA issuer and TMEM owner: per stage, scales -> TMEM, then 4 MMAs of K = 32
+//              into one of two fp32 accumulators in TMEM.
+//   warps 2-5  epilogue: TMEM -> registers, term pairs summed.  gate_up: a 128-row tile
+//              is 64 gate rows then the 64 matching up rows; the up half goes to the gate
+//              warps through shared memory, which apply the SwiGLU clamp and write h split
+//              again into two MXFP8 terms for the down GEMM.  down: rows scaled by the
+//              gate weight, written as fp32 in slot order for the combine.
+#include <algorithm>
+
+#include "kernels.cuh"
+#include "tcgen05.cuh"
+
+namespace fp4 {
+namespace {
+
+constexpr int kBsThreads = 6 * 32;
+constexpr int kBsMaxStages = 8;
+constexpr int kKT = 128;                  // K elements per stage (one 128-byte swizzle row of E4M3)
+constexpr int kATile = 128 * 128;         // shared bytes of the 128-row FP4 tile (16-byte slots)
+constexpr int kSfBytes = 512 + 1024;      // A scale atom + two B scale atoms per stage
+constexpr int kSfCols = 16;               // TMEM columns per stage for scales (A: 4, B: 8)
+constexpr int kMaxTokCap = 112;           // tokens per unit: 2 x 112 accumulator columns
+
+struct BsLayout {
+  int ntok_cap;      // tokens per work unit
+  int ncols;         // accumulator columns per buffer = rows of the B box (16-multiple)
+  int stage_bytes;
+  int stages;
+  int tmem_cols;
+  int xch_off, cnt_off, off_off, pre_off, bar_off;
+  int smem_bytes;
+};
+
+struct BsUnit {
+  int e, tile, slot0, ntok;
+};
+
+__device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* off, const int* pre, int E,
+                                            int tiles, int cap) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  BsUnit un;
+  un.e = lo;
+  const int n = cnt[lo];
+  const int groups = (n + cap - 1) / cap;
+  const int local = u - pre[lo];
+  un.tile = local / groups;
+  const int grp = local - un.tile * groups;
+  un.slot0 = off[lo] + grp * cap;
+  un.ntok = min(cap, n - grp * cap);
+  return un;
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on the mbarrier when this thread's earlier cp.async copies land (the pending
+// count is raised first, so the expected arrival count is unchanged).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// byte offset of scale row r (0..255) in the stage's B scale atoms, or of a weight row
+// (0..127) in the A atom: 32-row x 16-byte atoms, row r at lane r % 32, word (r / 32) % 4
+__device__ __forceinline__ uint32_t sf_row_off(int r) {
+  return static_cast<uint32_t>((r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4);
+}
+
+// E4M3 byte (satfinite, round to nearest even) of y, and its exact value
+__device__ __forceinline__ uint32_t e4m3_rn(float y, float& back) {
+  uint16_t pair;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(0.0f), "f"(y));
+  const uint32_t q = pair & 0xFFu;
+  uint32_t h2;
+  asm("{\n .reg .b16 lo;\n cvt.u16.u32 lo, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}" : "=r"(h2) : "r"(q));
+  back = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
+  return q;
+}
+
+// UE8M0 exponent for a block of E4M3 elements: the least e with amax * 2^-e <= 448
+// (E4M3's largest finite value), clamped to the UE8M0 range; 2^-127 for an all-zero block.
+__device__ __forceinline__ int e4m3_block_exp(float amax) {
+  if (!(amax > 0.f) || !isfinite(amax)) return -127;
+  int ex;
+  frexpf(amax, &ex);                        // amax = f 2^ex, f in [0.5, 1)
+  int e = ex - 9;                           // amax 2^-e in [256, 512)
+  if (ldexpf(amax, -e) > 448.f) e += 1;
+  return max(-127, min(127, e));
+}
+
+// Two-term split of the 32 values held by a warp (one per lane): E4M3 bytes of both
+// terms for this lane and the two UE8M0 scale bytes (identical in all lanes).
+__device__ __forceinline__ void warp_split2(float v, uint32_t& q1, uint32_t& q2, uint32_t& s1, uint32_t& s2) {
+  float amax = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const int e1 = e4m3_block_exp(amax);
+  float b1;
+  q1 = e4m3_rn(ldexpf(v, -e1), b1);
+  const float r = v - ldexpf(b1, e1);
+  float ramax = fabsf(r);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ramax = fmaxf(ramax, __shfl_xor_sync(0xFFFFFFFFu, ramax, o));
+  const int e2 = e4m3_block_exp(ramax);
+  float b2;
+  q2 = e4m3_rn(ldexpf(r, -e2), b2);
+  s1 = static_cast<uint32_t>(e1 + 127);
+  s2 = static_cast<uint32_t>(e2 + 127);
+}
+
+// x [T][H] bf16 -> slot-ordered two-term MXFP8 rows: q [2P][H] E4M3, s [2P][H/32] UE8M0,
+// rows 2i, 2i + 1 for slot i (token perm[i] / k).  One thread per 32-element block.
+__global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict__ x,
+                                                      const int32_t* __restrict__ perm, int k, int P, int H,
+                                                      uint8_t* __restrict__ q, uint8_t* __restrict__ s) {
+  pdl_wait();
+  const int nb = H / 32;
+  const int64_t total = static_cast<int64_t>(P) * nb;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int slot = static_cast<int>(idx / nb), b = static_cast<int>(idx % nb);
+    const int t = perm[slot] / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + 32 * b);
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 w = src[j];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[8 * j + 2 * i] = __uint_as_float(ws[i] << 16);
+        v[8 * j + 2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e1 = e4m3_block_exp(amax);
+    uint32_t w1[8], w2[8];
+    float ramax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float b1;
+      const uint32_t c = e4m3_rn(ldexpf(v[i], -e1), b1);
+      if ((i & 3) == 0) w1[i >> 2] = 0;
+      w1[i >> 2] |= c << (8 * (i & 3));
+      v[i] -= ldexpf(b1, e1);
+      ramax = fmaxf(ramax, fabsf(v[i]));
+    }
+    const int e2 = e4m3_block_exp(ramax);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float b2;
+      const uint32_t c = e4m3_rn(ldexpf(v[i], -e2), b2);
+      if ((i & 3) == 0) w2[i >> 2] = 0;
+      w2[i >> 2] |= c << (8 * (i & 3));
+    }
+    uint4* d1 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot)) * H + 32 * b);
+    uint4* d2 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot) + 1) * H + 32 * b);
+    d1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+    d2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+    d2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+    s[(2 * static_cast<int64_t>(slot)) * nb + b] = static_cast<uint8_t>(e1 + 127);
+    s[(2 * static_cast<int64_t>(slot) + 1) * nb + b] = static_cast<uint8_t>(e2 + 127);
+  }
+  pdl_launch_dependents();
+}
+
+template <int kEpi>
+__global__ void __launch_bounds__(kBsThreads, 1)
+    bs_moe_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const BsArgs a, const BsLayout L) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - sraw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = L.stages;
+  const uint32_t bar_full = sbase + L.bar_off;
+  const uint32_t bar_empty = bar_full + 8 * kBsMaxStages;
+  const uint32_t bar_accf = bar_empty + 8 * kBsMaxStages;    // [2] MMA done + unit id posted
+  const uint32_t bar_acce = bar_accf + 16;                    // [2] epilogue done with the buffer
+  const uint32_t bar_final = bar_acce + 16;
+  const uint32_t tmem_holder = bar_final + 8;
+  int* stage_unit = reinterpret_cast<int*>(smem + L.bar_off + 8 * (2 * kBsMaxStages + 5) + 8);
+  int* acc_unit = stage_unit + kBsMaxStages;
+  int* cnt = reinterpret_cast<int*>(smem + L.cnt_off);
+  int* off = reinterpret_cast<int*>(smem + L.off_off);
+  int* pre = reinterpret_cast<int*>(smem + L.pre_off);
+  const int E = a.E;
+  const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 64 : a.rows_per_expert / 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 2);
+      mbar_init(bar_acce + 8 * b, 4);
+    }
+    mbar_init(bar_final, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_holder, static_cast<uint32_t>(L.tmem_cols));
+    tc::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + (tmem_holder - sbase));
+  pdl_wait();
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) slot_begin(a.slot);
+
+  // per-expert unit prefix; units are ordered (expert, tile, token group)
+  for (int e = threadIdx.x; e < E; e += kBsThreads) cnt[e] = a.counts[e];
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int sc = 0, su = 0;
+    for (int e = e0; e < e1; ++e) {
+      sc += cnt[e];
+      su += (cnt[e] + L.ntok_cap - 1) / L.ntok_cap * tiles;
+    }
+    int ic = sc, iu = su;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vc = __shfl_up_sync(0xFFFFFFFFu, ic, o), vu = __shfl_up_sync(0xFFFFFFFFu, iu, o);
+      if (lane >= o) { ic += vc; iu += vu; }
+    }
+    int rc = ic - sc, ru = iu - su;
+    for (int e = e0; e < e1; ++e) {
+      off[e] = rc;
+      pre[e] = ru;
+      rc += cnt[e];
+      ru += (cnt[e] + L.ntok_cap - 1) / L.ntok_cap * tiles;
+    }
+    if (lane == 31) { off[E] = ic; pre[E] = iu; }
+  }
+  __syncthreads();
+  const int n_units = pre[E];
+  const int nk = a.K / kKT;
+  const int ksf = a.K / 32;             // scale bytes per row
+  const uint32_t stg = static_cast<uint32_t>(L.stage_bytes);
+
+  if (warp == 0) {
+    // ------------------------------------ producer ------------------------------------
+    int it = 0;
+    int u = blockIdx.x;
+    bool ok = true;
+    while (ok) {
+      if (u >= n_units) {
+        const int s = it % S;
+        if (it >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / S) & 1) ^ 1, a.status))) break;
+        if (lane == 0) {
+          stage_unit[s] = -1;
+          mbar_arrive(bar_full + 8 * s);
+        }
+        ++it;
+        break;
+      }
+      const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
+      const int64_t rbase = static_cast<int64_t>(un.e) * a.rows_per_expert;
+      const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 64 : rbase + un.tile * 128;
+      const int64_t y1 = (kEpi == kEpiSwiglu) ? rbase + a.inter + un.tile * 64 : y0 + 64;
+      const int brow0 = 2 * un.slot0, nrows = 2 * un.ntok;
+      for (int c = 0; c < nk; ++c, ++it) {
+        const int s = it % S;
+        if (it >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / S) & 1) ^ 1, a.status))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) stage_unit[s] = u;
+        const uint32_t st = sbase + s * stg;
+        const uint32_t sfa = st + kATile + L.ncols * kKT, sfb = sfa + 512;
+        const int kb = c * (kKT / 32);
+        for (int r = lane; r < 128; r += 32) {
+          const int64_t row = (r < 64) ? y0 + r : y1 + (r - 64);
+          cp_async4(sfa + sf_row_off(r), a.a_scales + row * ksf + kb);
+        }
+        for (int r = lane; r < nrows; r += 32)
+          cp_async4(sfb + sf_row_off(r), a.b_scales + static_cast<int64_t>(brow0 + r) * ksf + kb);
+        cp_async_mbar_arrive(bar_full + 8 * s);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(128 * kKT / 2 + L.ncols * kKT));
+          tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * s);
+          tma_load_2d(st + 64 * 128, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
+          tma_load_2d(st + kATile, &tmB, c * kKT, brow0, bar_full + 8 * s);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      int v = 0;
+      if (lane == 0) v = static_cast<int>(gridDim.x + atomicAdd(a.unit_next, 1u));
+      u = __shfl_sync(0xFFFFFFFFu, v, 0);
+    }
+    // every copy this warp started has landed before the CTA may exit
+    for (int d = 1; d <= S && d <= it; ++d) {
+      const int j = it - d;
+      mbar_wait(bar_full + 8 * (j % S), (j / S) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------ MMA issuer ----------------------------------
+    const uint32_t sf_t0 = tmem + static_cast<uint32_t>(2 * L.ncols);
+    int it = 0, uc = 0;
+    bool ok = true;
+    while (ok) {
+      const int s0 = it % S;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s0, (it / S) & 1, a.status))) break;
+      const int u = *reinterpret_cast<volatile int*>(&stage_unit[s0]);
+      const int buf = uc & 1;
+      if (uc >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_acce + 8 * buf, ((uc >> 1) & 1) ^ 1, a.status))) break;
+      if (lane == 0) {
+        acc_unit[buf] = u;
+        mbar_arrive(bar_accf + 8 * buf);
+        if (u < 0) mbar_arrive(bar_accf + 8 * buf);
+      }
+      __syncwarp();
+      if (u < 0) break;
+      tc::fence_after_sync();
+      const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
+      const uint32_t N = static_cast<uint32_t>((2 * un.ntok + 15) & ~15);
+      const uint32_t idesc = tc::idesc_mxf8f6f4(5u, 0u, 128u, N);
+      const uint32_t d_t = tmem + static_cast<uint32_t>(buf * L.ncols);
+      for (int c = 0; c < nk; ++c, ++it) {
+        const int s = it % S;
+        if (c > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s, (it / S) & 1, a.status))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        if (lane == 0) {
+          fence_proxy_async();    // scale bytes from cp.async, read next by the tensor-core copy
+          const uint32_t st = sbase + s * stg;
+          const uint32_t sfa = st + kATile + L.ncols * kKT, sfb = sfa + 512;
+          const uint32_t sfa_t = sf_t0 + s * kSfCols, sfb_t = sfa_t + 4;
+          tc::cp_sf_32x128b_x4(sfa_t, tc::desc_k_interleave(sfa));
+          tc::cp_sf_32x128b_x4(sfb_t, tc::desc_k_interleave(sfb));
+          if (N > 128) tc::cp_sf_32x128b_x4(sfb_t + 4, tc::desc_k_interleave(sfb + 512));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tc::mma_mxf8f6f4(d_t, tc::desc_k_sw128(st + 32 * j), tc::desc_k_sw128(st + kATile + 32 * j), idesc,
+                             sfa_t, sfb_t, static_cast<uint32_t>(j), static_cast<uint32_t>((c | j) != 0));
+          tc::commit(bar_empty + 8 * s);
+          if (c == nk - 1) tc::commit(bar_accf + 8 * buf);
+        }
+        __syncwarp();
+      }
+      ++uc;
+    }
+    // all MMAs of this thread complete before TMEM is released
+    if (lane == 0) tc::commit(bar_final);
+    __syncwarp();
+    mbar_wait(bar_final, 0, a.status);
+  } else {
+    // ------------------------------------ epilogue -------------------------------------
+    const int q = warp & 3;                    // TMEM lane quadrant this warp may access
+    const int row = 32 * q + lane;             // accumulator row = weight row of the tile
+    float* xch = reinterpret_cast<float*>(smem + L.xch_off);   // [2][64][8]
+    int uc = 0;
+    while (true) {
+      const int buf = uc & 1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_accf + 8 * buf, (uc >> 1) & 1, a.status))) break;
+      const int u = *reinterpret_cast<volatile int*>(&acc_unit[buf]);
+      if (u < 0) break;
+      tc::fence_after_sync();
+      const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
+      const uint32_t d_t = tmem + static_cast<uint32_t>(buf * L.ncols) + (static_cast<uint32_t>(32 * q) << 16);
+      const int N = (2 * un.ntok + 15) & ~15;
+      if (kEpi == kEpiSwiglu) {
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          float* xb = xch + ((c0 >> 4) & 1) * (64 * 8);
+          uint32_t v[16];
+          tc::ld_32x32b_x16(d_t + static_cast<uint32_t>(c0), v);
+          tc::ld_wait();
+          if (q >= 2) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              xb[(row - 64) * 8 + j] = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+          }
+          epi_bar_sync();
+          if (q < 2) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int i = (c0 >> 1) + j;
+              if (i < un.ntok) {                 // warp-uniform
+                const float g = fminf(__uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]), a.limit);
+                const float uu = fminf(fmaxf(xb[row * 8 + j], -a.limit), a.limit);
+                const float hv = g / (1.0f + expf(-g)) * uu;
+                uint32_t q1, q2, s1, s2;
+                warp_split2(hv, q1, q2, s1, s2);
+                const int64_t slot = un.slot0 + i;
+                const int64_t col = static_cast<int64_t>(un.tile) * 64 + row;
+                a.hq[(2 * slot) * a.inter + col] = static_cast<uint8_t>(q1);
+                a.hq[(2 * slot + 1) * a.inter + col] = static_cast<uint8_t>(q2);
+                if (lane == 0) {
+                  a.hs[(2 * slot) * (a.inter / 32) + col / 32] = static_cast<uint8_t>(s1);
+                  a.hs[(2 * slot + 1) * (a.inter / 32) + col / 32] = static_cast<uint8_t>(s2);
+                }
+              }
+            }
+          }
+        }
+      } else {
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          uint32_t v[16];
+          tc::ld_32x32b_x16(d_t + static_cast<uint32_t>(c0), v);
+          tc::ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = (c0 >> 1) + j;
+            if (i < un.ntok) {
+              const int64_t slot = un.slot0 + i;
+              const float wgt = a.gw[a.perm[slot]];
+              a.o_out[slot * a.ldo + static_cast<int64_t>(un.tile) * 128 + row] =
+                  (__uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1])) * wgt;
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      epi_bar_sync();
+      if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
+      ++uc;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, static_cast<uint32_t>(L.tmem_cols));
+  }
+  if (threadIdx.x == 0) slot_end(a.slot);
+}
+
+constexpr int kBsSmemLimit = 227 * 1024;
+
+bool bs_layout(int T, int E, BsLayout* L) {
+  L->ntok_cap = std::min(kMaxTokCap, (T + 7) / 8 * 8);
+  L->ncols = (2 * L->ntok_cap + 15) / 16 * 16;
+  L->stage_bytes = static_cast<int>(align_up(static_cast<size_t>(kATile + L->ncols * kKT + kSfBytes), 1024));
+  // fixed part (after the stages): exchange buffer, per-expert tables, barriers
+  int off = 0;
+  const int xch = off;
+  off += 2 * 64 * 8 * 4;
+  const int c0 = off;
+  off += 4 * (E + 1);
+  const int o0 = off;
+  off += 4 * (E + 1);
+  const int p0 = off;
+  off += 4 * (E + 1);
+  off = static_cast<int>(align_up(off, 16));
+  const int b0 = off;
+  off += 8 * (2 * kBsMaxStages + 5) + 8 + 4 * (kBsMaxStages + 2);
+  const int fixed = static_cast<int>(align_up(off, 16));
+  int S = (kBsSmemLimit - 1024 - fixed) / L->stage_bytes;
+  S = std::min(S, kBsMaxStages);
+  while (S > 0 && 2 * L->ncols + kSfCols * S > 512) --S;
+  if (S < 2) return false;
+  L->stages = S;
+  const int body = S * L->stage_bytes;
+  L->xch_off = body + xch;
+  L->cnt_off = body + c0;
+  L->off_off = body + o0;
+  L->pre_off = body + p0;
+  L->bar_off = body + b0;
+  L->smem_bytes = body + fixed + 1024;      // + slack for the 1024-byte alignment of the base
+  const int need = 2 * L->ncols + kSfCols * S;
+  int cols = 32;
+  while (cols < need) cols *= 2;
+  L->tmem_cols = cols;
+  return true;
+}
+
+}  // namespace
+
+fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, int k, int P, int H, uint8_t* q, uint8_t* s,
+                          cudaStream_t st) {
+  const int64_t total = static_cast<int64_t>(P) * (H / 32);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, num_sms() * 16)));
+  return launch_pdl(split_x_kernel, dim3(grid), dim3(256), 0, st, true, x, perm, k, P, H, q, s);
+}
+
+bool bs_supported(int T, int E, int H, int I) {
+  BsLayout L;
+  return H % kKT == 0 && I % kKT == 0 && I % 64 == 0 && H % 128 == 0 && bs_layout(T, E, &L);
+}
+
+fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
+  BsLayout L;
+  if (!bs_layout(T, a.E, &L)) return FP4_ERR_UNSUPPORTED;
+  CUtensorMap mA, mB;
+  FP4_TRY(make_tmap_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.codes, static_cast<uint64_t>(a.K),
+                       static_cast<uint64_t>(a.rows_total), static_cast<uint64_t>(a.K / 2), kKT, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+  FP4_TRY(make_tmap_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_q, static_cast<uint64_t>(a.K),
+                       static_cast<uint64_t>(2) * a.P, static_cast<uint64_t>(a.K), kKT,
+                       static_cast<uint32_t>(L.ncols), CU_TENSOR_MAP_SWIZZLE_128B));
+  auto kern = (a.epi == kEpiSwiglu) ? bs_moe_kernel<kEpiSwiglu> : bs_moe_kernel<kEpiDown>;
+  static thread_local bool configured[2] = {false, false};
+  const int which = (a.epi == kEpiSwiglu) ? 0 : 1;
+  if (!configured[which]) {
+    FP4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmemLimit));
+    configured[which] = true;
+  }
+  return launch_pdl(kern, dim3(num_sms()), dim3(kBsThreads), static_cast<size_t>(L.smem_bytes), st, true, mA,
+                    mB, a, L);
+}
+
+}  // namespace fp4

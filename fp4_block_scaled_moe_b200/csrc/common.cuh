@@ -54,6 +54,10 @@ int num_sms();                    // SM count of the current device (cached per 
 cudaError_t enable_pdl_attr(cudaLaunchAttribute* attr);
 
 // Tensor maps (TMA descriptors) via the driver entry point, no libcuda link needed.
+// inner_elems and box_inner count elements of dtype (for the 4-bit type, 4-bit elements).
+fp4_status make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner_elems,
+                        uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                        CUtensorMapSwizzle swz);
 fp4_status make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows,
                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
                            CUtensorMapSwizzle swz);

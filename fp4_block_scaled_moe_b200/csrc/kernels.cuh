@@ -102,4 +102,34 @@ __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __res
                                uint16_t* __restrict__ y);
 
 
+// Block-scaled tensor-core expert GEMM (MXFP4 weights x two-term MXFP8 activations).
+struct BsArgs {
+  int epi;                        // kEpiSwiglu (gate_up + SwiGLU) or kEpiDown
+  const uint8_t* codes;           // A: [rows_total][K/2] E2M1 pairs
+  const uint8_t* a_scales;        // A: [rows_total][K/32] UE8M0
+  int64_t rows_total;
+  int K;
+  int rows_per_expert;
+  int inter;                      // I (gate rows, then up rows, per expert)
+  int E;
+  int P;                          // routed slots T*k
+  const int32_t* counts;
+  const uint8_t* b_q;             // B: [2P][K] E4M3, rows 2i and 2i+1 = terms of slot i
+  const uint8_t* b_scales;        // B: [2P][K/32] UE8M0
+  float limit;
+  uint8_t* hq;                    // gate_up out: h terms [2P][I] E4M3
+  uint8_t* hs;                    //              [2P][I/32] UE8M0
+  const float* gw;                // down: gate weights by pair, perm: slot -> pair
+  const int32_t* perm;
+  float* o_out;                   // down out: [P][ldo] fp32, slot order
+  int ldo;
+  uint32_t* status;
+  KernelSlot* slot;
+  uint32_t* unit_next;
+};
+bool bs_supported(int T, int E, int H, int I);
+fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st);
+fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, int k, int P, int H, uint8_t* q, uint8_t* s,
+                          cudaStream_t st);
+
 }  // namespace fp4

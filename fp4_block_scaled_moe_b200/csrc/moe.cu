@@ -13,12 +13,23 @@ namespace {
 
 constexpr size_t kAlign = 256;
 
+enum Variant { kVarGemv = 1, kVarTensor = 2 };
+
+// Which expert-GEMM kernels a call runs (the arguments are already validated).
+int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
+  const bool tc_ok = w->fmt == FP4_MXFP4 && bs_supported(T, w->num_experts, w->hidden, w->inter);
+  if (w->kernel_variant == kVarTensor) return kVarTensor;
+  if (w->kernel_variant == kVarGemv) return kVarGemv;
+  return (tc_ok && static_cast<int64_t>(T) * k >= 4 * static_cast<int64_t>(w->num_experts)) ? kVarTensor : kVarGemv;
+}
+
 struct MoeWs {
-  size_t status, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, h, o, total;
+  size_t status, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, h, o, xq, xs, hq, hs, total;
 };
 
 bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   const int64_t E = w->num_experts, H = w->hidden, I = w->inter;
+  const bool tensor = moe_variant(w, T, k) == kVarTensor;
   const int64_t P = static_cast<int64_t>(T) * k;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -35,9 +46,14 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   L->perm = take(sizeof(int32_t) * P);
   L->inv = take(sizeof(int32_t) * P);
   L->sexp = take(sizeof(int32_t) * T);
-  L->x16 = take(sizeof(uint16_t) * T * H);
-  L->h = take(sizeof(uint16_t) * P * I);
+  L->x16 = take(tensor ? 0 : sizeof(uint16_t) * T * H);
+  L->h = take(tensor ? 0 : sizeof(uint16_t) * P * I);
   L->o = take(sizeof(float) * P * H);
+  // tensor-core variant: x and h as two MXFP8 terms per slot (rows 2i, 2i + 1)
+  L->xq = take(tensor ? 2 * P * H : 0);
+  L->xs = take(tensor ? 2 * P * (H / 32) : 0);
+  L->hq = take(tensor ? 2 * P * I : 0);
+  L->hs = take(tensor ? 2 * P * (I / 32) : 0);
   L->total = off;
   return true;
 }
@@ -65,6 +81,9 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (!(w->swiglu_limit > 0.f) || !(w->swiglu_limit <= 128.f)) return FP4_ERR_INVALID_ARG;
   if (!w->gu_codes || !w->gu_scales || !w->dn_codes || !w->dn_scales) return FP4_ERR_INVALID_ARG;
   if (w->fmt == FP4_NVFP4 && (!w->gu_tscale || !w->dn_tscale)) return FP4_ERR_INVALID_ARG;
+  if (w->kernel_variant < 0 || w->kernel_variant > 2) return FP4_ERR_INVALID_ARG;
+  if (w->kernel_variant == kVarTensor && !(w->fmt == FP4_MXFP4 && bs_supported(T, E, H, I)))
+    return FP4_ERR_UNSUPPORTED;
   if (!aligned16(w->gu_codes) || !aligned16(w->gu_scales) || !aligned16(w->dn_codes) || !aligned16(w->dn_scales))
     return FP4_ERR_ALIGNMENT;
   return FP4_OK;
@@ -115,6 +134,56 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   ra.x16 = reinterpret_cast<__half*>(ws + L.x16);
   ra.sexp = reinterpret_cast<int*>(ws + L.sexp);
   ra.ctrl = reinterpret_cast<WsControl*>(ws + L.status);
+  if (moe_variant(w, T, k) == kVarTensor) {
+    ra.x16 = nullptr;
+    ra.logits_only = false;
+    ra.pdl_first = true;
+    FP4_TRY(launch_route(ra, st));
+    uint8_t* xq = ws + L.xq;
+    uint8_t* xs = ws + L.xs;
+    FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, k, P, H, xq, xs, st));
+    BsArgs g{};
+    g.epi = kEpiSwiglu;
+    g.codes = w->gu_codes;
+    g.a_scales = w->gu_scales;
+    g.rows_total = static_cast<int64_t>(E) * 2 * I;
+    g.K = H;
+    g.rows_per_expert = 2 * I;
+    g.inter = I;
+    g.E = E;
+    g.P = P;
+    g.counts = ra.counts;
+    g.b_q = xq;
+    g.b_scales = xs;
+    g.limit = w->swiglu_limit;
+    g.hq = ws + L.hq;
+    g.hs = ws + L.hs;
+    g.status = &ra.ctrl->status;
+    g.slot = &ra.ctrl->slot[0];
+    g.unit_next = &ra.ctrl->unit_next[0];
+    FP4_TRY(launch_bs(g, T, st));
+    BsArgs d = g;
+    d.epi = kEpiDown;
+    d.codes = w->dn_codes;
+    d.a_scales = w->dn_scales;
+    d.rows_total = static_cast<int64_t>(E) * H;
+    d.K = I;
+    d.rows_per_expert = H;
+    d.b_q = g.hq;
+    d.b_scales = g.hs;
+    d.gw = ra.gw;
+    d.perm = ra.perm;
+    d.o_out = reinterpret_cast<float*>(ws + L.o);
+    d.ldo = H;
+    d.slot = &ra.ctrl->slot[1];
+    d.unit_next = &ra.ctrl->unit_next[1];
+    FP4_TRY(launch_bs(d, T, st));
+    const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
+    const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, num_sms() * 8));
+    return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, true, static_cast<const float*>(d.o_out),
+                      static_cast<const int32_t*>(ra.inv), T, k, H, static_cast<uint16_t*>(y_bf16));
+  }
+
   // small routing problems finish inside the gate_up kernel's prologue
   const bool fused = P <= kRouteMaxPairs && E <= kRouteMaxExperts;
   ra.logits_only = fused;

@@ -156,6 +156,11 @@ typedef struct fp4_moe_weights {
   const int32_t* dn_rowptr;
   const int32_t* dn_col;
   const uint16_t* dn_val;
+  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores for MXFP4 when T*k >= 4E,
+   * i.e. four or more tokens per expert on average), 1 = CUDA-core grouped GEMV,
+   * 2 = block-scaled tensor-core GEMM (MXFP4 only; FP4_ERR_UNSUPPORTED otherwise).
+   * Any other value is FP4_ERR_INVALID_ARG. */
+  int32_t kernel_variant;
 } fp4_moe_weights;
 
 /* Optional copies of the routing results of a forward call (each pointer may be NULL). */
@@ -184,7 +189,10 @@ size_t moe_fp4_workspace_size(const fp4_moe_weights* w, int32_t T, int32_t k);
  * route: optional host struct of device pointers receiving the routing results.
  * Accuracy: float32 accumulation of exactly dequantised weights; against a float64
  * evaluation of the same definition, rel. Frobenius error <= 5e-3 and per-element
- * |err| <= 2e-2 (|ref| + 1).
+ * |err| <= 2e-2 (|ref| + 1).  The tensor-core variant (MXFP4) feeds x and h to the
+ * MMA as two E4M3 terms per value with a power-of-two scale per 32 (residual about
+ * 2^-8 of each value); the CUDA-core variant feeds them as float16 with a per-row
+ * power-of-two scale.
  */
 fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
                            const float* router_bias, int32_t T, int32_t k, void* y_bf16,

@@ -85,6 +85,17 @@ def test_forward_named_refusals():
     assert fwd(_weights(fmt=L.FP4_CB4)) == 5
     assert fwd(_weights(E=1 << 20, H=1 << 16, I=1 << 16)) == 3
     assert fwd(_weights(), ws=None) == 6
+    bad = _weights()
+    bad.kernel_variant = 7
+    assert fwd(bad) == 1                       # unknown kernel variant
+    nv = _weights(fmt=L.FP4_NVFP4)
+    nv.kernel_variant = 2
+    assert fwd(nv) == 5                        # tensor-core variant is MXFP4 only
+    small_w, big_w = _weights(), _weights()
+    small_w.kernel_variant, big_w.kernel_variant = 1, 2
+    # the tensor-core variant keeps x and h as two-term E4M3 rows in the workspace
+    assert lib.moe_fp4_workspace_size(ctypes.byref(big_w), 4, 2) != lib.moe_fp4_workspace_size(
+        ctypes.byref(small_w), 4, 2)
     assert fwd(_weights(), nbytes=100) == 6
     w = _weights()
     assert lib.moe_fp4_workspace_size(ctypes.byref(w), 4, 2) > 0
