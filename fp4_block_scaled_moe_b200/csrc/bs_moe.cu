@@ -9,17 +9,23 @@
 // 2^-8 |x| per element.  The two terms of token slot i are B rows 2i and 2i + 1, so the
 // product with x_i is D[:, 2i] + D[:, 2i + 1].
 //
+// A work unit is (expert, tile, token group): two 128-row weight tiles A0 and A1 times
+// the group's activation rows, into two fp32 accumulators D0 and D1 in TMEM.  gate_up:
+// A0 = gate rows t*128.., A1 = the up rows of the same intermediate indices, so g and u
+// of one index sit in the same TMEM lane.  down: A0, A1 = output rows t*256.. and
+// t*256+128...
+//
 // Warp roles of one persistent CTA per SM:
-//   warp 0     producer: TMA of the weight tile (FP4 widened to 16-byte slots, 128-byte
-//              swizzle) and of the activation-term tile; 4-byte async copies place the
-//              scale bytes in the 32-row x 16-byte atoms the TMEM scale copy reads.
-//   warp 1     MMA issuer and TMEM owner: per stage, scales -> TMEM, then 4 MMAs of K = 32
-//              into one of two fp32 accumulators in TMEM.
-//   warps 2-5  epilogue: TMEM -> registers, term pairs summed.  gate_up: a 128-row tile
-//              is 64 gate rows then the 64 matching up rows; the up half goes to the gate
-//              warps through shared memory, which apply the SwiGLU clamp and write h split
-//              again into two MXFP8 terms for the down GEMM.  down: rows scaled by the
-//              gate weight, written as fp32 in slot order for the combine.
+//   warp 0     producer: TMA of the two weight tiles (FP4 widened to 16-byte slots,
+//              128-byte swizzle) and of the activation-term tile; 4-byte async copies
+//              place the scale bytes in the 32-row x 16-byte atoms the TMEM scale copy
+//              reads.
+//   warp 1     MMA issuer and TMEM owner: per stage, scales -> TMEM, then 2 x 4 MMAs of
+//              K = 32 into one of two double-buffered accumulator pairs.
+//   warps 2-5  epilogue, one TMEM lane quadrant each: term pairs summed; gate_up applies
+//              the SwiGLU clamp and writes h split again into two MXFP8 terms for the
+//              down GEMM; down scales rows by the gate weight and writes fp32 in slot
+//              order for the combine.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -31,18 +37,18 @@ namespace {
 constexpr int kBsThreads = 6 * 32;
 constexpr int kBsMaxStages = 8;
 constexpr int kKT = 128;                  // K elements per stage (one 128-byte swizzle row of E4M3)
-constexpr int kATile = 128 * 128;         // shared bytes of the 128-row FP4 tile (16-byte slots)
-constexpr int kSfBytes = 512 + 1024;      // A scale atom + two B scale atoms per stage
-constexpr int kSfCols = 16;               // TMEM columns per stage for scales (A: 4, B: 8)
-constexpr int kMaxTokCap = 112;           // tokens per unit: 2 x 112 accumulator columns
+constexpr int kATile = 128 * 128;         // shared bytes of one 128-row FP4 tile (16-byte slots)
+constexpr int kSfBytes = 3 * 512;         // scale atoms per stage: A0, A1, B
+constexpr int kSfCols = 16;               // TMEM columns per stage for scales (4 each)
+constexpr int kMaxTokCap = 56;            // tokens per unit: accumulators of 2 x 56 columns
 
 struct BsLayout {
   int ntok_cap;      // tokens per work unit
-  int ncols;         // accumulator columns per buffer = rows of the B box (16-multiple)
+  int ncols;         // columns per accumulator = rows of the B box (16-multiple, <= 112)
   int stage_bytes;
   int stages;
   int tmem_cols;
-  int xch_off, cnt_off, off_off, pre_off, bar_off;
+  int cnt_off, off_off, pre_off, bar_off;
   int smem_bytes;
 };
 
@@ -77,12 +83,11 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// byte offset of scale row r (0..255) in the stage's B scale atoms, or of a weight row
-// (0..127) in the A atom: 32-row x 16-byte atoms, row r at lane r % 32, word (r / 32) % 4
+// byte offset of row r (0..127) in a scale atom: 32 rows x 16 bytes, row r at line r % 32,
+// word r / 32 (the four bytes of a word are the four 32-element blocks of one stage)
 __device__ __forceinline__ uint32_t sf_row_off(int r) {
-  return static_cast<uint32_t>((r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4);
+  return static_cast<uint32_t>((r & 31) * 16 + (r >> 5) * 4);
 }
 
 // E4M3 byte (satfinite, round to nearest even) of y, and its exact value
@@ -96,33 +101,33 @@ __device__ __forceinline__ uint32_t e4m3_rn(float y, float& back) {
   return q;
 }
 
-// UE8M0 exponent for a block of E4M3 elements: the least e with amax * 2^-e <= 448
-// (E4M3's largest finite value), clamped to the UE8M0 range; 2^-127 for an all-zero block.
+// UE8M0 exponent for a block of E4M3 elements from the bits of its amax (finite, >= 0):
+// the least e with amax * 2^-e <= 448 (E4M3's largest finite value), kept in [-126, 127]
+// so that 2^e and 2^-e are normal floats.  amax in [2^(B-127), 2^(B-126)) for biased
+// exponent B; e = B - 135 puts amax 2^-e in [256, 512), one more when the significand
+// exceeds 1.75.
 __device__ __forceinline__ int e4m3_block_exp(float amax) {
-  if (!(amax > 0.f) || !isfinite(amax)) return -127;
-  int ex;
-  frexpf(amax, &ex);                        // amax = f 2^ex, f in [0.5, 1)
-  int e = ex - 9;                           // amax 2^-e in [256, 512)
-  if (ldexpf(amax, -e) > 448.f) e += 1;
-  return max(-127, min(127, e));
+  const uint32_t b = __float_as_uint(amax);
+  const int e = static_cast<int>(b >> 23) - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return max(-126, min(127, e));
+}
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
+
+// max |v| over the warp: for non-negative floats the bit patterns order like the values
+__device__ __forceinline__ float warp_amax(float v) {
+  return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fabsf(v))));
 }
 
 // Two-term split of the 32 values held by a warp (one per lane): E4M3 bytes of both
 // terms for this lane and the two UE8M0 scale bytes (identical in all lanes).
 __device__ __forceinline__ void warp_split2(float v, uint32_t& q1, uint32_t& q2, uint32_t& s1, uint32_t& s2) {
-  float amax = fabsf(v);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-  const int e1 = e4m3_block_exp(amax);
+  const int e1 = e4m3_block_exp(warp_amax(v));
   float b1;
-  q1 = e4m3_rn(ldexpf(v, -e1), b1);
-  const float r = v - ldexpf(b1, e1);
-  float ramax = fabsf(r);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ramax = fmaxf(ramax, __shfl_xor_sync(0xFFFFFFFFu, ramax, o));
-  const int e2 = e4m3_block_exp(ramax);
+  q1 = e4m3_rn(v * exp2i(-e1), b1);
+  const float r = v - b1 * exp2i(e1);
+  const int e2 = e4m3_block_exp(warp_amax(r));
   float b2;
-  q2 = e4m3_rn(ldexpf(r, -e2), b2);
+  q2 = e4m3_rn(r * exp2i(-e2), b2);
   s1 = static_cast<uint32_t>(e1 + 127);
   s2 = static_cast<uint32_t>(e2 + 127);
 }
@@ -155,22 +160,24 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
     const int e1 = e4m3_block_exp(amax);
+    const float inv1 = exp2i(-e1), up1 = exp2i(e1);
     uint32_t w1[8], w2[8];
     float ramax = 0.f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       float b1;
-      const uint32_t c = e4m3_rn(ldexpf(v[i], -e1), b1);
+      const uint32_t c = e4m3_rn(v[i] * inv1, b1);
       if ((i & 3) == 0) w1[i >> 2] = 0;
       w1[i >> 2] |= c << (8 * (i & 3));
-      v[i] -= ldexpf(b1, e1);
+      v[i] -= b1 * up1;
       ramax = fmaxf(ramax, fabsf(v[i]));
     }
     const int e2 = e4m3_block_exp(ramax);
+    const float inv2 = exp2i(-e2);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       float b2;
-      const uint32_t c = e4m3_rn(ldexpf(v[i], -e2), b2);
+      const uint32_t c = e4m3_rn(v[i] * inv2, b2);
       if ((i & 3) == 0) w2[i >> 2] = 0;
       w2[i >> 2] |= c << (8 * (i & 3));
     }
@@ -208,7 +215,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   int* off = reinterpret_cast<int*>(smem + L.off_off);
   int* pre = reinterpret_cast<int*>(smem + L.pre_off);
   const int E = a.E;
-  const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 64 : a.rows_per_expert / 128;
+  const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 128 : a.rows_per_expert / 256;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -269,6 +276,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   const int nk = a.K / kKT;
   const int ksf = a.K / 32;             // scale bytes per row
   const uint32_t stg = static_cast<uint32_t>(L.stage_bytes);
+  const uint32_t b_off = 2 * kATile, sf_off = 2 * kATile + L.ncols * kKT;   // within a stage
 
   if (warp == 0) {
     // ------------------------------------ producer ------------------------------------
@@ -288,9 +296,12 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       }
       const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
       const int64_t rbase = static_cast<int64_t>(un.e) * a.rows_per_expert;
-      const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 64 : rbase + un.tile * 128;
-      const int64_t y1 = (kEpi == kEpiSwiglu) ? rbase + a.inter + un.tile * 64 : y0 + 64;
+      const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 128 : rbase + un.tile * 256;
+      const int64_t y1 = (kEpi == kEpiSwiglu) ? y0 + a.inter : y0 + 128;
       const int brow0 = 2 * un.slot0, nrows = 2 * un.ntok;
+      const uint8_t* sa0 = a.a_scales + y0 * ksf;
+      const uint8_t* sa1 = a.a_scales + y1 * ksf;
+      const uint8_t* sb = a.b_scales + static_cast<int64_t>(brow0) * ksf;
       for (int c = 0; c < nk; ++c, ++it) {
         const int s = it % S;
         if (it >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / S) & 1) ^ 1, a.status))) {
@@ -299,21 +310,22 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         }
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st = sbase + s * stg;
-        const uint32_t sfa = st + kATile + L.ncols * kKT, sfb = sfa + 512;
+        const uint32_t sf = st + sf_off;
         const int kb = c * (kKT / 32);
-        for (int r = lane; r < 128; r += 32) {
-          const int64_t row = (r < 64) ? y0 + r : y1 + (r - 64);
-          cp_async4(sfa + sf_row_off(r), a.a_scales + row * ksf + kb);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;
+          cp_async4(sf + sf_row_off(r), sa0 + static_cast<int64_t>(r) * ksf + kb);
+          cp_async4(sf + 512 + sf_row_off(r), sa1 + static_cast<int64_t>(r) * ksf + kb);
         }
-        for (int r = lane; r < nrows; r += 32)
-          cp_async4(sfb + sf_row_off(r), a.b_scales + static_cast<int64_t>(brow0 + r) * ksf + kb);
+        for (int r = lane; r < nrows; r += 32) cp_async4(sf + 1024 + sf_row_off(r), sb + static_cast<int64_t>(r) * ksf + kb);
         cp_async_mbar_arrive(bar_full + 8 * s);
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(128 * kKT / 2 + L.ncols * kKT));
+          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(2 * 128 * kKT / 2 + L.ncols * kKT));
           tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * s);
-          tma_load_2d(st + 64 * 128, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
-          tma_load_2d(st + kATile, &tmB, c * kKT, brow0, bar_full + 8 * s);
+          tma_load_2d(st + kATile, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
+          tma_load_2d(st + b_off, &tmB, c * kKT, brow0, bar_full + 8 * s);
         }
         __syncwarp();
       }
@@ -329,7 +341,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------ MMA issuer ----------------------------------
-    const uint32_t sf_t0 = tmem + static_cast<uint32_t>(2 * L.ncols);
+    const uint32_t sf_t0 = tmem + static_cast<uint32_t>(4 * L.ncols);
     int it = 0, uc = 0;
     bool ok = true;
     while (ok) {
@@ -349,7 +361,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
       const uint32_t N = static_cast<uint32_t>((2 * un.ntok + 15) & ~15);
       const uint32_t idesc = tc::idesc_mxf8f6f4(5u, 0u, 128u, N);
-      const uint32_t d_t = tmem + static_cast<uint32_t>(buf * L.ncols);
+      const uint32_t d0 = tmem + static_cast<uint32_t>(buf * 2 * L.ncols), d1 = d0 + static_cast<uint32_t>(L.ncols);
       for (int c = 0; c < nk; ++c, ++it) {
         const int s = it % S;
         if (c > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s, (it / S) & 1, a.status))) {
@@ -360,15 +372,19 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         if (lane == 0) {
           fence_proxy_async();    // scale bytes from cp.async, read next by the tensor-core copy
           const uint32_t st = sbase + s * stg;
-          const uint32_t sfa = st + kATile + L.ncols * kKT, sfb = sfa + 512;
-          const uint32_t sfa_t = sf_t0 + s * kSfCols, sfb_t = sfa_t + 4;
-          tc::cp_sf_32x128b_x4(sfa_t, tc::desc_k_interleave(sfa));
-          tc::cp_sf_32x128b_x4(sfb_t, tc::desc_k_interleave(sfb));
-          if (N > 128) tc::cp_sf_32x128b_x4(sfb_t + 4, tc::desc_k_interleave(sfb + 512));
+          const uint32_t sf = st + sf_off;
+          const uint32_t t0 = sf_t0 + s * kSfCols;
+          tc::cp_sf_32x128b_x4(t0, tc::desc_k_interleave(sf));
+          tc::cp_sf_32x128b_x4(t0 + 4, tc::desc_k_interleave(sf + 512));
+          tc::cp_sf_32x128b_x4(t0 + 8, tc::desc_k_interleave(sf + 1024));
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tc::mma_mxf8f6f4(d_t, tc::desc_k_sw128(st + 32 * j), tc::desc_k_sw128(st + kATile + 32 * j), idesc,
-                             sfa_t, sfb_t, static_cast<uint32_t>(j), static_cast<uint32_t>((c | j) != 0));
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t bd = tc::desc_k_sw128(st + b_off + 32 * j);
+            const uint32_t acc = static_cast<uint32_t>((c | j) != 0);
+            tc::mma_mxf8f6f4(d0, tc::desc_k_sw128(st + 32 * j), bd, idesc, t0, t0 + 8, static_cast<uint32_t>(j), acc);
+            tc::mma_mxf8f6f4(d1, tc::desc_k_sw128(st + kATile + 32 * j), bd, idesc, t0 + 4, t0 + 8,
+                             static_cast<uint32_t>(j), acc);
+          }
           tc::commit(bar_empty + 8 * s);
           if (c == nk - 1) tc::commit(bar_accf + 8 * buf);
         }
@@ -383,8 +399,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   } else {
     // ------------------------------------ epilogue -------------------------------------
     const int q = warp & 3;                    // TMEM lane quadrant this warp may access
-    const int row = 32 * q + lane;             // accumulator row = weight row of the tile
-    float* xch = reinterpret_cast<float*>(smem + L.xch_off);   // [2][64][8]
+    const int row = 32 * q + lane;             // accumulator row within each 128-row tile
     int uc = 0;
     while (true) {
       const int buf = uc & 1;
@@ -393,61 +408,61 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       if (u < 0) break;
       tc::fence_after_sync();
       const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
-      const uint32_t d_t = tmem + static_cast<uint32_t>(buf * L.ncols) + (static_cast<uint32_t>(32 * q) << 16);
+      const uint32_t d0 =
+          tmem + static_cast<uint32_t>(buf * 2 * L.ncols) + (static_cast<uint32_t>(32 * q) << 16);
+      const uint32_t d1 = d0 + static_cast<uint32_t>(L.ncols);
       const int N = (2 * un.ntok + 15) & ~15;
       if (kEpi == kEpiSwiglu) {
+        const int64_t col = static_cast<int64_t>(un.tile) * 128 + row;
+        const int64_t scol = col >> 5;
         for (int c0 = 0; c0 < N; c0 += 16) {
-          float* xb = xch + ((c0 >> 4) & 1) * (64 * 8);
-          uint32_t v[16];
-          tc::ld_32x32b_x16(d_t + static_cast<uint32_t>(c0), v);
+          uint32_t vg[16], vu[16];
+          tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), vg);
+          tc::ld_32x32b_x16(d1 + static_cast<uint32_t>(c0), vu);
           tc::ld_wait();
-          if (q >= 2) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              xb[(row - 64) * 8 + j] = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
-          }
-          epi_bar_sync();
-          if (q < 2) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int i = (c0 >> 1) + j;
-              if (i < un.ntok) {                 // warp-uniform
-                const float g = fminf(__uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]), a.limit);
-                const float uu = fminf(fmaxf(xb[row * 8 + j], -a.limit), a.limit);
-                const float hv = g / (1.0f + expf(-g)) * uu;
-                uint32_t q1, q2, s1, s2;
-                warp_split2(hv, q1, q2, s1, s2);
-                const int64_t slot = un.slot0 + i;
-                const int64_t col = static_cast<int64_t>(un.tile) * 64 + row;
-                a.hq[(2 * slot) * a.inter + col] = static_cast<uint8_t>(q1);
-                a.hq[(2 * slot + 1) * a.inter + col] = static_cast<uint8_t>(q2);
-                if (lane == 0) {
-                  a.hs[(2 * slot) * (a.inter / 32) + col / 32] = static_cast<uint8_t>(s1);
-                  a.hs[(2 * slot + 1) * (a.inter / 32) + col / 32] = static_cast<uint8_t>(s2);
-                }
+          for (int j = 0; j < 8; ++j) {
+            const int i = (c0 >> 1) + j;
+            const float g = fminf(__uint_as_float(vg[2 * j]) + __uint_as_float(vg[2 * j + 1]), a.limit);
+            const float uu = fminf(fmaxf(__uint_as_float(vu[2 * j]) + __uint_as_float(vu[2 * j + 1]), -a.limit), a.limit);
+            const float hv = __fdividef(g, 1.0f + __expf(-g)) * uu;
+            uint32_t q1, q2, s1, s2;
+            warp_split2(hv, q1, q2, s1, s2);
+            if (i < un.ntok) {
+              const int64_t r0 = 2 * (static_cast<int64_t>(un.slot0) + i);
+              a.hq[r0 * a.inter + col] = static_cast<uint8_t>(q1);
+              a.hq[(r0 + 1) * a.inter + col] = static_cast<uint8_t>(q2);
+              if (lane == 0) {
+                a.hs[r0 * (a.inter / 32) + scol] = static_cast<uint8_t>(s1);
+                a.hs[(r0 + 1) * (a.inter / 32) + scol] = static_cast<uint8_t>(s2);
               }
             }
           }
         }
       } else {
+        // gate weights of the unit's tokens, one per lane (ntok <= 64)
+        const float w_lo = (lane < un.ntok) ? a.gw[a.perm[un.slot0 + lane]] : 0.f;
+        const float w_hi = (lane + 32 < un.ntok) ? a.gw[a.perm[un.slot0 + 32 + lane]] : 0.f;
+        float* o0 = a.o_out + static_cast<int64_t>(un.slot0) * a.ldo + static_cast<int64_t>(un.tile) * 256 + row;
         for (int c0 = 0; c0 < N; c0 += 16) {
-          uint32_t v[16];
-          tc::ld_32x32b_x16(d_t + static_cast<uint32_t>(c0), v);
+          uint32_t v0[16], v1[16];
+          tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), v0);
+          tc::ld_32x32b_x16(d1 + static_cast<uint32_t>(c0), v1);
           tc::ld_wait();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int i = (c0 >> 1) + j;
+            const float wgt = __shfl_sync(0xFFFFFFFFu, (i < 32) ? w_lo : w_hi, i & 31);
             if (i < un.ntok) {
-              const int64_t slot = un.slot0 + i;
-              const float wgt = a.gw[a.perm[slot]];
-              a.o_out[slot * a.ldo + static_cast<int64_t>(un.tile) * 128 + row] =
-                  (__uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1])) * wgt;
+              float* o = o0 + static_cast<int64_t>(i) * a.ldo;
+              o[0] = (__uint_as_float(v0[2 * j]) + __uint_as_float(v0[2 * j + 1])) * wgt;
+              o[128] = (__uint_as_float(v1[2 * j]) + __uint_as_float(v1[2 * j + 1])) * wgt;
             }
           }
         }
       }
       tc::fence_before_sync();
-      epi_bar_sync();
+      __syncwarp();
       if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
       ++uc;
     }
@@ -466,11 +481,9 @@ constexpr int kBsSmemLimit = 227 * 1024;
 bool bs_layout(int T, int E, BsLayout* L) {
   L->ntok_cap = std::min(kMaxTokCap, (T + 7) / 8 * 8);
   L->ncols = (2 * L->ntok_cap + 15) / 16 * 16;
-  L->stage_bytes = static_cast<int>(align_up(static_cast<size_t>(kATile + L->ncols * kKT + kSfBytes), 1024));
-  // fixed part (after the stages): exchange buffer, per-expert tables, barriers
+  L->stage_bytes = static_cast<int>(align_up(static_cast<size_t>(2 * kATile + L->ncols * kKT + kSfBytes), 1024));
+  // fixed part (after the stages): per-expert tables, barriers
   int off = 0;
-  const int xch = off;
-  off += 2 * 64 * 8 * 4;
   const int c0 = off;
   off += 4 * (E + 1);
   const int o0 = off;
@@ -483,17 +496,16 @@ bool bs_layout(int T, int E, BsLayout* L) {
   const int fixed = static_cast<int>(align_up(off, 16));
   int S = (kBsSmemLimit - 1024 - fixed) / L->stage_bytes;
   S = std::min(S, kBsMaxStages);
-  while (S > 0 && 2 * L->ncols + kSfCols * S > 512) --S;
+  while (S > 0 && 4 * L->ncols + kSfCols * S > 512) --S;
   if (S < 2) return false;
   L->stages = S;
   const int body = S * L->stage_bytes;
-  L->xch_off = body + xch;
   L->cnt_off = body + c0;
   L->off_off = body + o0;
   L->pre_off = body + p0;
   L->bar_off = body + b0;
   L->smem_bytes = body + fixed + 1024;      // + slack for the 1024-byte alignment of the base
-  const int need = 2 * L->ncols + kSfCols * S;
+  const int need = 4 * L->ncols + kSfCols * S;
   int cols = 32;
   while (cols < need) cols *= 2;
   L->tmem_cols = cols;
@@ -511,7 +523,7 @@ fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, int k, int P, 
 
 bool bs_supported(int T, int E, int H, int I) {
   BsLayout L;
-  return H % kKT == 0 && I % kKT == 0 && I % 64 == 0 && H % 128 == 0 && bs_layout(T, E, &L);
+  return H % 256 == 0 && I % 128 == 0 && bs_layout(T, E, &L);
 }
 
 fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
@@ -519,7 +531,7 @@ fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
   if (!bs_layout(T, a.E, &L)) return FP4_ERR_UNSUPPORTED;
   CUtensorMap mA, mB;
   FP4_TRY(make_tmap_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.codes, static_cast<uint64_t>(a.K),
-                       static_cast<uint64_t>(a.rows_total), static_cast<uint64_t>(a.K / 2), kKT, 64,
+                       static_cast<uint64_t>(a.rows_total), static_cast<uint64_t>(a.K / 2), kKT, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B));
   FP4_TRY(make_tmap_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_q, static_cast<uint64_t>(a.K),
                        static_cast<uint64_t>(2) * a.P, static_cast<uint64_t>(a.K), kKT,
