@@ -59,6 +59,29 @@ def per_expert_bytes(cfg):
     return b, gu // 2 + gu // B + (4 if cfg.fmt == "nvfp4" else 0)
 
 
+def is_prefill(cfg):
+    return "prefill" in cfg.name
+
+
+def uses_tensor_cores(cfg):
+    """The library's automatic kernel choice: tensor cores for MXFP4 at >= 4 tokens per expert."""
+    return cfg.fmt == "mxfp4" and cfg.T * cfg.k >= 4 * cfg.E
+
+
+def layer_flops(cfg, tokens=None):
+    """Dense-equivalent flops of the routed experts: 2 T k (2I H + H I) = 6 T k H I."""
+    T = cfg.T if tokens is None else tokens
+    return 6 * T * cfg.k * cfg.H * cfg.I
+
+
+def work_per_step(cfg, counts, tokens=None):
+    """Amount of the metric's work in one step and its rate unit: prefill counts
+    TFLOP, decode counts GB of algorithmic bytes."""
+    if is_prefill(cfg):
+        return layer_flops(cfg, tokens) / 1e12, "TFLOP/s"
+    return algorithmic_bytes(cfg, counts, tokens) / 1e9, "GB/s"
+
+
 def algorithmic_bytes(cfg, counts, tokens=None):
     """Active-bytes rule: every routed expert's weight bytes once + router + x + y."""
     per, _ = per_expert_bytes(cfg)
@@ -172,6 +195,7 @@ def run_ours(args, cfg, rank, world):
         step(0)
     torch.cuda.synchronize()
     counts = route["counts"].cpu().numpy()
+    work_step, _ = work_per_step(cfg, counts)
     bytes_step = algorithmic_bytes(cfg, counts)
     # one CUDA graph per weight copy (kernel launches replayed without host overhead)
     graphs = []
@@ -247,7 +271,8 @@ def run_ours(args, cfg, rank, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total, e2e_ms, gu_ms, dn_ms = t.tolist()
     kern_ms = {"gate_up": gu_ms, "down": dn_ms, "launches": kern["gate_up_launches"]}
-    return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, e2e_ms=e2e_ms / args.steps,
+    return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, work_step=work_step,
+                e2e_ms=e2e_ms / args.steps,
                 kern=kern, kern_ms=kern_ms, clocks=clocks, copies=copies, counts=counts, status=status,
                 h2d=T * cfg.H * 2, d2h=T * cfg.H * 2, launches_per_step=launches_per_step)
 
@@ -276,18 +301,34 @@ def oracle_sample(cfg, n_tokens):
     def run():
         M.moe_layer(xf[tok], wr, bias, cfg.k, bank, cfg.swiglu_limit)
 
-    return run, algorithmic_bytes(cfg, counts, tokens=n_tokens)
+    return run, work_per_step(cfg, counts, tokens=n_tokens)[0]
 
 
 def roofline(cfg, r, hbm_peak, peaks):
-    """Dominant kernel: gate_up with the fused SwiGLU. Algorithmic bytes per launch =
+    """Dominant kernel: gate_up with the fused SwiGLU, timed per launch on the device.
+    Prefill: algorithmic flops per launch 4 T k H I against the measured bf16 peak (the
+    two-term E4M3 x E2M1 MMAs run at the FP8 rate, twice the MMA work of one bf16 pass,
+    so the bf16 rate is their ceiling for these flops).
+    Decode: algorithmic bytes per launch =
     codes + scales of the gate_up rows of every routed expert + the f16 activation rows
     read once per unit + h written; duration = its device time per launch in the timed region."""
+    ms = r["kern_ms"]["gate_up"]
+    if is_prefill(cfg):
+        flops = 4 * cfg.T * cfg.k * cfg.H * cfg.I
+        ach = flops / (ms * 1e-3) / 1e12 if ms > 0 else None
+        peak = peaks.get("bf16_tflops", 1590.0)
+        return {"kernel": "bs_moe_kernel<gate_up+swiglu>", "bound": "tensor", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": (ach / peak) if ach else None, "traffic": None,
+                "peak_source": ("MEASURED_PEAKS.json bf16_tflops, burst (of measured)" if "bf16_tflops" in peaks
+                                else "fallback 1590 TFLOP/s bf16 (of fallback)"),
+                "frac_of_sustained": (ach / peaks["bf16_tflops_sustained"]) if ach and "bf16_tflops_sustained" in peaks
+                else None,
+                "flops_per_launch": int(flops), "ms_per_launch": ms, "down_ms_per_launch": r["kern_ms"]["down"],
+                "timer": "device globaltimer per launch, accumulated in the workspace over the timed steps"}
     _, gu_per_expert = per_expert_bytes(cfg)
     d = int(np.count_nonzero(r["counts"]))
     P = cfg.T * cfg.k
     alg = d * gu_per_expert + cfg.T * cfg.H * 2 + P * cfg.I * 2
-    ms = r["kern_ms"]["gate_up"]
     ach = alg / (ms * 1e-3) / 1e9 if ms > 0 else None
     return {"kernel": "decode_kernel<gate_up+swiglu>", "bound": "hbm", "achieved": ach, "peak": hbm_peak,
             "unit": "GB/s", "frac": (ach / hbm_peak) if ach else None, "traffic": None,
@@ -300,8 +341,8 @@ def cpu_baseline(cfg, budget_s=20.0):
     """The float64 oracle timed on this host's cores on a bounded sample of the same
     workload: the layer for the first tokens (all their routed experts), repeated until
     about budget_s of CPU time; value in the metric's unit (algorithmic GB/s)."""
-    n_tok = min(cfg.T, 4)
-    run, sample_bytes = oracle_sample(cfg, n_tok)
+    n_tok = 1 if is_prefill(cfg) else min(cfg.T, 4)
+    run, sample_work = oracle_sample(cfg, n_tok)
     run()                                            # warm (dequantise caches, BLAS threads)
     reps, t0 = 0, time.perf_counter()
     while True:
@@ -311,7 +352,8 @@ def cpu_baseline(cfg, budget_s=20.0):
         if dt > budget_s or reps >= 50:
             break
     per = dt / reps
-    return {"value": sample_bytes / per / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+    return {"value": sample_work / per, "unit": work_per_step(cfg, np.ones(1))[1], "cores": blas_threads(),
+            "kind": "oracle",
             "sample": f"first {n_tok} of {cfg.T} tokens with all their routed experts, float64 numpy, "
                       f"{reps} repetitions in {dt:.1f} s", "ms_per_sample": per * 1e3}
 
@@ -336,21 +378,22 @@ def main():
         if rank != 0:
             return
         n_tok = 1
-        run, sample_bytes = oracle_sample(cfg, n_tok)
+        run, sample_work = oracle_sample(cfg, n_tok)
+        unit = work_per_step(cfg, np.ones(1))[1]
         for _ in range(args.warmup):
             run()
         t0 = time.perf_counter()
         for _ in range(args.steps):
             run()
         dt = (time.perf_counter() - t0) / args.steps
-        v = sample_bytes / dt / 1e9
-        line = {"impl": "reference", "metric": metric, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        v = sample_work / dt
+        line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": workload, "sample": f"{n_tok} token(s) of {cfg.T}, all their experts"},
-                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                "cpu_baseline": {"value": v, "unit": unit, "cores": blas_threads(), "kind": "oracle",
                                  "sample": f"{n_tok} token(s) of {cfg.T}, float64 numpy oracle"},
-                "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
 
@@ -365,17 +408,29 @@ def main():
     except OSError:
         pass
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    value = r["bytes_step"] * world / (r["ms_per_step"] * 1e-3) / 1e9
+    unit = work_per_step(cfg, r["counts"])[1]
+    value = r["work_step"] * world / (r["ms_per_step"] * 1e-3)
+    bank_mb = r["copies"] * per_expert_bytes(cfg)[0] * cfg.E / 1e6
+    conf = {"workload": workload, "tokens": cfg.T, "experts": cfg.E, "hidden": cfg.H, "inter": cfg.I,
+            "top_k": cfg.k, "format": cfg.fmt, "parallelism": f"replicas{world}",
+            "l2": (f"weights rotate over {r['copies']} copies ({bank_mb:.0f} MB) > L2" if r["copies"] > 1
+                   else f"weights {bank_mb:.0f} MB > L2, one copy"),
+            "distinct_experts": int(np.count_nonzero(r["counts"])),
+            "expert_kernels": "tensor-core block-scaled" if uses_tensor_cores(cfg) else "CUDA-core grouped GEMV",
+            "bytes_per_step": int(r["bytes_step"])}
+    if is_prefill(cfg):
+        conf["tokens_per_s"] = cfg.T * world / (r["ms_per_step"] * 1e-3)
+        conf["pct_of_bf16_measured_peak"] = 100 * value / world / peaks.get("bf16_tflops", 1590.0)
+        conf["pct_of_fp4_dense_nominal_9000"] = 100 * value / world / 9000.0
+    else:
+        conf["pct_of_hbm_peak"] = 100 * value / world / hbm_peak
     line = {
-        "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16xe2m1->f32", "data": "synthetic",
-        "config": {"workload": workload, "tokens": cfg.T, "experts": cfg.E, "hidden": cfg.H, "inter": cfg.I,
-                   "top_k": cfg.k, "format": cfg.fmt, "parallelism": f"replicas{world}",
-                   "l2": f"weights rotate over {r['copies']} copies ({r['copies'] * per_expert_bytes(cfg)[0] * cfg.E / 1e6:.0f} MB) > L2",
-                   "distinct_experts": int(np.count_nonzero(r["counts"])),
-                   "bytes_per_step": int(r["bytes_step"]), "pct_of_hbm_peak": 100 * value / world / hbm_peak},
-        "e2e": {"value": r["bytes_step"] * world / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
+        "vs_baseline": None, "dtype": "e4m3x2xe2m1->f32" if uses_tensor_cores(cfg) else "f16xe2m1->f32",
+        "data": "synthetic",
+        "config": conf,
+        "e2e": {"value": r["work_step"] * world / (r["e2e_ms"] * 1e-3), "unit": unit,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "roofline": roofline(cfg, r, hbm_peak, peaks),

@@ -269,11 +269,199 @@ __global__ void __launch_bounds__(1024) perm_kernel(const int32_t* __restrict__ 
   pdl_launch_dependents();
 }
 
+// ---- R1 for many tokens: tensor-core tiles -------------------------------------------
+// logits = x Wr^T + bias with x exactly bf16 and Wr float32 split exactly (to 2^-24 of
+// each weight) into three bf16 terms, hi + mid + lo; bf16 x bf16 products are exact and
+// accumulate in float32 on the tensor cores (mma.sync m16n8k16).  CTA tile: 128 tokens x
+// 64 experts, K chunks of 32, two shared-memory stages; 8 warps of 32 x 32.
+constexpr int kLgBM = 128, kLgBN = 64, kLgBK = 32, kLgLd = kLgBK + 8;   // row pitch 80 B
+constexpr int kLgStage = (kLgBM + 3 * kLgBN) * kLgLd * 2;                // bytes per stage
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9},"
+      " {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// bf16 (round to nearest even) of v and the exact remainder v - bf16(v)
+__device__ __forceinline__ uint32_t bf16_split(float v, float& rest) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  rest = v - __bfloat162float(h);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(h));
+}
+
+__global__ void __launch_bounds__(256) logits_mma_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
+                                                         const float* __restrict__ bias, int T, int H, int E,
+                                                         float* __restrict__ logits, WsControl* __restrict__ ctrl) {
+  extern __shared__ __align__(16) uint8_t lg_smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp & 3, wn = warp >> 2;
+  const int t0 = blockIdx.x * kLgBM, e0 = blockIdx.y * kLgBN;
+  const uint32_t sb = smem_u32(lg_smem);
+  // loader assignment: x tile 128 rows x 4 chunks of 16 B; W tile 64 rows x 8 float4
+  auto x_src = [&](int kt, int i) {
+    const int c = tid + 256 * i, r = c >> 2, ch = c & 3;
+    const int tr = min(t0 + r, T - 1);
+    return x + static_cast<int64_t>(tr) * H + kt * kLgBK + ch * 8;
+  };
+  auto x_dst = [&](int stage, int i) {
+    const int c = tid + 256 * i, r = c >> 2, ch = c & 3;
+    return sb + stage * kLgStage + (r * kLgLd + ch * 8) * 2;
+  };
+  float4 wv[2];
+  auto w_load = [&](int kt) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + 256 * i, r = c >> 3, ch = c & 7;
+      const int er = min(e0 + r, E - 1);
+      wv[i] = *reinterpret_cast<const float4*>(wr + static_cast<int64_t>(er) * H + kt * kLgBK + ch * 4);
+    }
+  };
+  auto w_store = [&](int stage) {
+    uint16_t* base = reinterpret_cast<uint16_t*>(lg_smem + stage * kLgStage) + kLgBM * kLgLd;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + 256 * i, r = c >> 3, ch = c & 7;
+      const float v[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+      uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float r1, r2, r3;
+        hi[j] = bf16_split(v[j], r1);
+        mid[j] = bf16_split(r1, r2);
+        lo[j] = bf16_split(r2, r3);
+      }
+      const int o = r * kLgLd + ch * 4;
+      *reinterpret_cast<uint2*>(base + o) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+      *reinterpret_cast<uint2*>(base + kLgBN * kLgLd + o) = make_uint2(mid[0] | (mid[1] << 16), mid[2] | (mid[3] << 16));
+      *reinterpret_cast<uint2*>(base + 2 * kLgBN * kLgLd + o) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+    }
+  };
+
+  const int nk = H / kLgBK;
+  w_load(0);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) cp_async16(x_dst(0, i), x_src(0, i));
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  pdl_wait();
+  if (ctrl != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) {
+    if (threadIdx.x == 0) ctrl->status = 0u;
+    ctrl->unit_next[threadIdx.x] = 0u;
+    KernelSlot* s = &ctrl->slot[threadIdx.x];
+    s->start_min = ~0ull;
+    s->end_max = 0ull;
+    s->done = 0u;
+  }
+  w_store(0);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+
+  float acc[2][4][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
+
+  for (int kt = 0; kt < nk; ++kt) {
+    const int cur = kt & 1;
+    if (kt + 1 < nk) {
+      w_load(kt + 1);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) cp_async16(x_dst(cur ^ 1, i), x_src(kt + 1, i));
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const uint32_t xs = sb + cur * kLgStage, ws = xs + kLgBM * kLgLd * 2;
+    // this chunk's products accumulate on the tensor cores from zero; the running sums
+    // take them with IEEE float adds, which bounds the tensor-core rounding to one chunk
+    float part[2][4][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) part[i][j][c] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < kLgBK; kk += 16) {
+      uint32_t af[2][4];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int row = wm * 32 + i * 16 + (lane & 15), col = kk + (lane >> 4) * 8;
+        ldsm_x4(xs + (row * kLgLd + col) * 2, af[i][0], af[i][1], af[i][2], af[i][3]);
+      }
+#pragma unroll
+      for (int term = 0; term < 3; ++term) {
+#pragma unroll
+        for (int jp = 0; jp < 2; ++jp) {
+          const int n = wn * 32 + jp * 16 + (lane & 7) + ((lane >> 4) << 3), col = kk + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(ws + ((term * kLgBN + n) * kLgLd + col) * 2, b0, b1, b2, b3);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            mma_bf16_16816(part[i][2 * jp], af[i], b0, b1);
+            mma_bf16_16816(part[i][2 * jp + 1], af[i], b2, b3);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][j][c] += part[i][j][c];
+    if (kt + 1 < nk) {
+      w_store(cur ^ 1);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
+    __syncthreads();
+  }
+  pdl_launch_dependents();
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = e0 + wn * 32 + j * 8 + 2 * tq;
+    const float b_0 = (bias != nullptr && e < E) ? bias[e] : 0.f;
+    const float b_1 = (bias != nullptr && e + 1 < E) ? bias[e + 1] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0 + wm * 32 + i * 16 + g + 8 * h;
+        if (t < T) {
+          float* out = logits + static_cast<int64_t>(t) * E;
+          if (e < E) out[e] = acc[i][j][2 * h] + b_0;
+          if (e + 1 < E) out[e + 1] = acc[i][j][2 * h + 1] + b_1;
+        }
+      }
+    }
+  }
+}
+
 size_t perm_smem_bytes(int E) { return (32 * static_cast<size_t>(E) + E + 1 + 1024) * sizeof(int32_t); }
 
 fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
   const int P = a.T * a.k;
-  if (a.logits_in == nullptr) {
+  if (a.logits_in == nullptr && a.x16 == nullptr && a.T >= 256 && a.H % kLgBK == 0) {
+    static thread_local bool configured = false;
+    if (!configured) {
+      FP4_TRY_CUDA(cudaFuncSetAttribute(logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * kLgStage));
+      configured = true;
+    }
+    dim3 grid((a.T + kLgBM - 1) / kLgBM, (a.E + kLgBN - 1) / kLgBN);
+    FP4_TRY(launch_pdl(logits_mma_kernel, grid, dim3(256), static_cast<size_t>(2 * kLgStage), st, a.pdl_first,
+                       static_cast<const uint16_t*>(a.x), a.router_w, a.router_bias, a.T, a.H, a.E, a.logits,
+                       a.ctrl));
+  } else if (a.logits_in == nullptr) {
     dim3 grid(a.E, (a.T + kTokGroup - 1) / kTokGroup);
     FP4_TRY(launch_pdl(logits_kernel, grid, dim3(kLogitsWarps * 32), 0, st, a.pdl_first,
                        static_cast<const uint16_t*>(a.x), a.router_w, a.router_bias, a.T, a.H, a.E,

@@ -37,7 +37,11 @@ def test_route_given_logits_bit_exact(T, E, k):
     assert np.allclose(got["topk_w"], w, rtol=2e-6, atol=1e-7)
 
 
-@pytest.mark.parametrize("cfg", [C.MOE_C2, C.MOE_C3], ids=["c2", "c3"])
+# C4 (8192 tokens) and a ragged shape take the tensor-core logits kernel (T >= 256)
+_RAGGED = C.MoEConfig("route_ragged_t300_e40", "mxfp4", T=300, E=40, H=544, I=256, k=3, zipf_bias=True)
+
+
+@pytest.mark.parametrize("cfg", [C.MOE_C2, C.MOE_C3, C.MOE_C4, _RAGGED], ids=["c2", "c3", "c4", "ragged_t300_e40"])
 def test_route_from_x(cfg):
     x_bits = D.activations_bf16(cfg.seed, cfg.T, cfg.H)
     wr = D.router_weights(cfg.seed, cfg.E, cfg.H)
