@@ -44,15 +44,21 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=C.MOE_C2.name, choices=sorted(C.FULL))
+    ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2],
+                    help="expert kernels: 0 chosen by the library, 1 CUDA-core GEMV, 2 tensor cores (MXFP4)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed CPU oracle sample")
     return ap.parse_args()
 
 
 def per_expert_bytes(cfg):
-    B = 32 if cfg.fmt == "mxfp4" else 16
+    """Dense bytes of one expert (all matrices, gate_up only): codes + scales; CB4 counts
+    indices + fp16 codebooks here and its CSR per expert separately (cb4_extra_bytes)."""
     gu = 2 * cfg.I * cfg.H
     dn = cfg.H * cfg.I
+    if cfg.fmt == "cb4":
+        return (gu + dn) // 2 + (gu + dn) // 4, gu // 2 + gu // 4
+    B = 32 if cfg.fmt == "mxfp4" else 16
     b = (gu + dn) // 2 + (gu + dn) // B
     if cfg.fmt == "nvfp4":
         b += 8
@@ -63,8 +69,10 @@ def is_prefill(cfg):
     return "prefill" in cfg.name
 
 
-def uses_tensor_cores(cfg):
-    """The library's automatic kernel choice: tensor cores for MXFP4 at >= 4 tokens per expert."""
+def uses_tensor_cores(cfg, variant=0):
+    """The library's kernel choice: tensor cores for MXFP4 at >= 4 tokens per expert."""
+    if variant:
+        return variant == 2
     return cfg.fmt == "mxfp4" and cfg.T * cfg.k >= 4 * cfg.E
 
 
@@ -74,21 +82,34 @@ def layer_flops(cfg, tokens=None):
     return 6 * T * cfg.k * cfg.H * cfg.I
 
 
-def work_per_step(cfg, counts, tokens=None):
+def work_per_step(cfg, counts, tokens=None, extra=None):
     """Amount of the metric's work in one step and its rate unit: prefill counts
     TFLOP, decode counts GB of algorithmic bytes."""
     if is_prefill(cfg):
         return layer_flops(cfg, tokens) / 1e12, "TFLOP/s"
-    return algorithmic_bytes(cfg, counts, tokens) / 1e9, "GB/s"
+    return algorithmic_bytes(cfg, counts, tokens, extra) / 1e9, "GB/s"
 
 
-def algorithmic_bytes(cfg, counts, tokens=None):
-    """Active-bytes rule: every routed expert's weight bytes once + router + x + y."""
+def cb4_extra_bytes(w):
+    """CB4 sparse term per expert: (gate_up, all) bytes of CSR values, columns and row
+    pointers, from the packed weights."""
+    out = []
+    for rp, rows in ((w.gu_rowptr, 2 * w.I), (w.dn_rowptr, w.H)):
+        r = rp.cpu().numpy().astype(np.int64)
+        nnz = r[rows::rows] - r[:-1:rows][:w.E]
+        out.append(nnz * 6 + 4 * rows)
+    return out[0], out[0] + out[1]
+
+
+def algorithmic_bytes(cfg, counts, tokens=None, extra=None):
+    """Active-bytes rule: every routed expert's weight bytes once + router + x + y
+    (extra: per-expert bytes beyond the dense part, counted for routed experts)."""
     per, _ = per_expert_bytes(cfg)
     d = int(np.count_nonzero(counts))
     T = cfg.T if tokens is None else tokens
     router = cfg.E * cfg.H * 4 + (cfg.E * 4 if cfg.zipf_bias else 0)
-    return d * per + router + 2 * T * cfg.H * 2
+    more = 0 if extra is None else int(np.sum(np.asarray(extra)[np.asarray(counts) > 0]))
+    return d * per + more + router + 2 * T * cfg.H * 2
 
 
 # ------------------------------------------------------------------------------------
@@ -151,15 +172,14 @@ def build_layer(cfg, copies, device):
     import torch
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from helpers import device_weights
+    import dataclasses
     weights = [device_weights(cfg, device=device)]
     for _ in range(copies - 1):
         w0 = weights[0]
-        clone = {n: (None if getattr(w0, n) is None else getattr(w0, n).clone())
-                 for n in ("gu_codes", "gu_scales", "dn_codes", "dn_scales", "gu_tscale", "dn_tscale")}
-        from fp4_block_scaled_moe_b200 import MoEWeights
-        weights.append(MoEWeights(cfg.fmt, cfg.E, cfg.H, cfg.I, clone["gu_codes"], clone["gu_scales"],
-                                  clone["dn_codes"], clone["dn_scales"], clone["gu_tscale"], clone["dn_tscale"],
-                                  cfg.swiglu_limit))
+        # an independent copy of every device tensor (codes, scales, codebooks, CSR)
+        weights.append(dataclasses.replace(w0, **{f.name: getattr(w0, f.name).clone()
+                                                  for f in dataclasses.fields(w0)
+                                                  if isinstance(getattr(w0, f.name), torch.Tensor)}))
     x_bits = D.activations_bf16(cfg.seed, cfg.T, cfg.H)
     wr = D.router_weights(cfg.seed, cfg.E, cfg.H)
     bias = D.zipf_bias(cfg.seed, cfg.E) if cfg.zipf_bias else None
@@ -179,6 +199,8 @@ def run_ours(args, cfg, rank, world):
     bank_bytes = per * cfg.E
     copies = max(2, int(np.ceil(2 * L2_BYTES / bank_bytes)) + 1) if bank_bytes < 4 * L2_BYTES else 1
     weights, x, wr, bias, x_bits = build_layer(cfg, copies, device)
+    for w in weights:
+        w.kernel_variant = args.variant
     structs = [w.c_struct() for w in weights]
     T, k = cfg.T, cfg.k
     ws_bytes = api.moe_fp4_workspace_size(weights[0], T, k)
@@ -195,8 +217,11 @@ def run_ours(args, cfg, rank, world):
         step(0)
     torch.cuda.synchronize()
     counts = route["counts"].cpu().numpy()
-    work_step, _ = work_per_step(cfg, counts)
-    bytes_step = algorithmic_bytes(cfg, counts)
+    extra_gu = extra_all = None
+    if cfg.fmt == "cb4":
+        extra_gu, extra_all = cb4_extra_bytes(weights[0])
+    work_step, _ = work_per_step(cfg, counts, extra=extra_all)
+    bytes_step = algorithmic_bytes(cfg, counts, extra=extra_all)
     # one CUDA graph per weight copy (kernel launches replayed without host overhead)
     graphs = []
     for c in range(copies):
@@ -271,7 +296,7 @@ def run_ours(args, cfg, rank, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total, e2e_ms, gu_ms, dn_ms = t.tolist()
     kern_ms = {"gate_up": gu_ms, "down": dn_ms, "launches": kern["gate_up_launches"]}
-    return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, work_step=work_step,
+    return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, work_step=work_step, extra_gu=extra_gu,
                 e2e_ms=e2e_ms / args.steps,
                 kern=kern, kern_ms=kern_ms, clocks=clocks, copies=copies, counts=counts, status=status,
                 h2d=T * cfg.H * 2, d2h=T * cfg.H * 2, launches_per_step=launches_per_step)
@@ -297,14 +322,20 @@ def oracle_sample(cfg, n_tokens):
         bank.packed("gu", int(e))
         bank.packed("dn", int(e))
     counts = np.bincount(ids.reshape(-1), minlength=cfg.E)
+    extra = None
+    if cfg.fmt == "cb4":            # CSR bytes of the sampled experts, from the oracle's own fits
+        extra = np.zeros(cfg.E, dtype=np.int64)
+        for e in np.unique(ids):
+            for which, rows in (("gu", 2 * cfg.I), ("dn", cfg.H)):
+                extra[e] += 6 * int(bank.packed(which, int(e))["row_ptr"][-1]) + 4 * rows
 
     def run():
         M.moe_layer(xf[tok], wr, bias, cfg.k, bank, cfg.swiglu_limit)
 
-    return run, work_per_step(cfg, counts, tokens=n_tokens)[0]
+    return run, work_per_step(cfg, counts, tokens=n_tokens, extra=extra)[0]
 
 
-def roofline(cfg, r, hbm_peak, peaks):
+def roofline(cfg, r, hbm_peak, peaks, tensor=False):
     """Dominant kernel: gate_up with the fused SwiGLU, timed per launch on the device.
     Prefill: algorithmic flops per launch 4 T k H I against the measured bf16 peak (the
     two-term E4M3 x E2M1 MMAs run at the FP8 rate, twice the MMA work of one bf16 pass,
@@ -329,8 +360,10 @@ def roofline(cfg, r, hbm_peak, peaks):
     d = int(np.count_nonzero(r["counts"]))
     P = cfg.T * cfg.k
     alg = d * gu_per_expert + cfg.T * cfg.H * 2 + P * cfg.I * 2
+    if r.get("extra_gu") is not None:
+        alg += int(np.sum(r["extra_gu"][r["counts"] > 0]))
     ach = alg / (ms * 1e-3) / 1e9 if ms > 0 else None
-    return {"kernel": "decode_kernel<gate_up+swiglu>", "bound": "hbm", "achieved": ach, "peak": hbm_peak,
+    return {"kernel": "bs_moe_kernel<gate_up+swiglu>" if tensor else "decode_kernel<gate_up+swiglu>", "bound": "hbm", "achieved": ach, "peak": hbm_peak,
             "unit": "GB/s", "frac": (ach / hbm_peak) if ach else None, "traffic": None,
             "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if "hbm_gbs" in peaks else "fallback",
             "bytes_per_launch": int(alg), "ms_per_launch": ms, "down_ms_per_launch": r["kern_ms"]["down"],
@@ -416,7 +449,7 @@ def main():
             "l2": (f"weights rotate over {r['copies']} copies ({bank_mb:.0f} MB) > L2" if r["copies"] > 1
                    else f"weights {bank_mb:.0f} MB > L2, one copy"),
             "distinct_experts": int(np.count_nonzero(r["counts"])),
-            "expert_kernels": "tensor-core block-scaled" if uses_tensor_cores(cfg) else "CUDA-core grouped GEMV",
+            "expert_kernels": "tensor-core block-scaled" if uses_tensor_cores(cfg, args.variant) else "CUDA-core grouped GEMV",
             "bytes_per_step": int(r["bytes_step"])}
     if is_prefill(cfg):
         conf["tokens_per_s"] = cfg.T * world / (r["ms_per_step"] * 1e-3)
@@ -427,13 +460,14 @@ def main():
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3x2xe2m1->f32" if uses_tensor_cores(cfg) else "f16xe2m1->f32",
+        "vs_baseline": None, "dtype": ("e4m3x2xe2m1->f32" if uses_tensor_cores(cfg, args.variant)
+                  else ("f16(codebook)xf16->f32" if cfg.fmt == "cb4" else "f16xe2m1->f32")),
         "data": "synthetic",
         "config": conf,
         "e2e": {"value": r["work_step"] * world / (r["e2e_ms"] * 1e-3), "unit": unit,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
-        "roofline": roofline(cfg, r, hbm_peak, peaks),
+        "roofline": roofline(cfg, r, hbm_peak, peaks, uses_tensor_cores(cfg, args.variant)),
         "clocks": r["clocks"],
         "device_status": r["status"],
     }

@@ -9,6 +9,7 @@ from .api import (  # noqa: F401
     fp4_launch_count,
     fp4_linear,
     fp4_pack,
+    fp4_pack_cb4,
     fp4_unpack,
     fp4_workspace_kernel_stats,
     fp4_workspace_status,

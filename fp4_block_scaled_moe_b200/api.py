@@ -58,6 +58,30 @@ def fp4_pack(w: torch.Tensor, fmt="mxfp4"):
     return codes, scales, ts
 
 
+def fp4_pack_cb4(w: torch.Tensor, threshold: float, mu: float = 0.0):
+    """CB4 pack of w [rows, k] (float32 or bf16): returns dict(idx, cb, row_ptr, col, val)
+    (see fp4_cb4_row_ptr / fp4_pack_cb4 in include/fp4moe.h)."""
+    lib = L.load()
+    _need(w, "w")
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("w must be float32 or bfloat16")
+    w2 = w.reshape(-1, w.shape[-1])
+    rows, k = w2.shape
+    dt = L.FP4_F32 if w.dtype == torch.float32 else L.FP4_BF16
+    dev = w.device
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    L.check("fp4_cb4_row_ptr", lib.fp4_cb4_row_ptr(_ptr(w2), dt, rows, k, float(threshold), float(mu), _ptr(row_ptr),
+                                                   _stream(dev)))
+    nnz = int(row_ptr[-1].item())
+    idx = torch.empty((rows, k // 2), dtype=torch.uint8, device=dev)
+    cb = torch.empty((rows, k // 128, 16), dtype=torch.int16, device=dev)
+    col = torch.empty(max(nnz, 1), dtype=torch.int32, device=dev)
+    val = torch.empty(max(nnz, 1), dtype=torch.int16, device=dev)
+    L.check("fp4_pack_cb4", lib.fp4_pack_cb4(_ptr(w2), dt, rows, k, float(threshold), float(mu), _ptr(row_ptr),
+                                             _ptr(idx), _ptr(cb), _ptr(col), _ptr(val), _stream(dev)))
+    return {"idx": idx, "cb": cb, "row_ptr": row_ptr, "col": col[:nnz], "val": val[:nnz]}
+
+
 def fp4_unpack(codes, scales, tensor_scale=None, fmt="mxfp4", out_dtype=torch.float32):
     lib = L.load()
     f = fmt_code(fmt)

@@ -13,6 +13,11 @@
 // fixed order and a fused epilogue writes the SwiGLU-with-clamp activation (gate_up),
 // the gate-weighted expert output (down) or y (dense layer).
 //
+// CB4 ("XFP：质量地板驱动的自适应码本量化", V2 dense + sparse): the 4-bit indices stream
+// like E2M1 codes; each row's fp16 codebooks for the stage arrive by one bulk copy; a
+// warp looks entries up in registers (low and high byte tables of the 16 entries,
+// byte-permute selection) and the CSR outlier term joins in the epilogue.
+//
 // In kModeRoute the gate_up kernel also finishes the router in its prologue: every CTA
 // takes the top-k of the logits, the per-expert counts and the stable permutation into
 // shared memory (CTA 0 also stores them for the later kernels), so no separate launch
@@ -134,12 +139,42 @@ __device__ __forceinline__ int64_t unit_row(const DecodeArgs& a, const Unit& un,
   return base + static_cast<int64_t>(un.tile) * kRows + r;
 }
 
+// CB4: eight 4-bit indices (low nibble first) -> four f16x2 registers of codebook
+// entries, from byte tables lo[q] / hi[q] holding the low / high bytes of entries
+// 4q .. 4q+3.  Byte-permute selects with the low three index bits among entries 0-7 and
+// 8-15; a mask made by sign-replicating each index's bit 3 picks between the two.
+// PTX prmt in its default mode: a selector nibble with bit 3 set replicates the sign bit
+// of the selected byte over the whole result byte (the CUDA intrinsic __byte_perm only
+// defines the low three selector bits).
+__device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ void cb4_lookup8(uint32_t w, const uint32_t (&lo)[4], const uint32_t (&hi)[4],
+                                            uint32_t (&h)[4]) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t v = half ? (w >> 16) : (w & 0xFFFFu);
+    const uint32_t sel = v & 0x7777u;
+    const uint32_t r = __byte_perm(v, 0u, 0x1100);                  // bytes B0 B0 B1 B1
+    const uint32_t sgn = (r & 0xFF00FF00u) | ((r << 4) & 0x00FF00FFu);   // bit 3 of nibble i -> bit 7 of byte i
+    const uint32_t msk = prmt_sx(sgn, 0u, 0xBA98u);                 // byte i = 0xFF where index i >= 8
+    const uint32_t la = __byte_perm(lo[0], lo[1], sel), lb = __byte_perm(lo[2], lo[3], sel);
+    const uint32_t ha = __byte_perm(hi[0], hi[1], sel), hb = __byte_perm(hi[2], hi[3], sel);
+    const uint32_t L = (la & ~msk) | (lb & msk), H = (ha & ~msk) | (hb & msk);
+    h[2 * half] = __byte_perm(L, H, 0x5140);
+    h[2 * half + 1] = __byte_perm(L, H, 0x7362);
+  }
+}
+
 template <int kFmt, int kEpi, int kMode, int KC>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a, const Layout L) {
   // stage geometry (must match make_layout)
   constexpr int kB = (kFmt == FP4_MXFP4) ? 32 : 16;
-  constexpr int kScaleRow = KC / kB;                 // scale bytes per row per stage
+  constexpr int kScaleRow = (kFmt == FP4_CB4) ? KC / 4 : KC / kB;   // scale (codebook) bytes per row per stage
   constexpr int kScalesOff = kRows * KC / 2;
   constexpr int kXOff = kScalesOff + kRows * kScaleRow;
   constexpr int kXRow = 2 * KC + 64;                 // padded f16 token row
@@ -280,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int64_t y0 = unit_row<kEpi>(a, un, 0), y1 = unit_row<kEpi>(a, un, 32);
       int xr = 0;
       if (lane < un.ntok) xr = (kEpi == kEpiSwiglu) ? perm_at(un.slot0 + lane) / a.topk : un.slot0 + lane;
-      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2);
+      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2 +
+                                                (kFmt == FP4_CB4 ? kRows * kScaleRow : 0));
       constexpr int words = kScaleRow / 4;
       for (int c = 0; c < L.nchunks; ++c, ++it) {
         const int s = it % L.stages;
@@ -292,15 +328,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st_base = sbase + s * L.stage_bytes;
         const int k0 = c * KC;
-        for (int w = lane; w < kRows * words; w += 32) {
-          const int r = w / words, cw = w - r * words;
-          const uint8_t* src = a.scales + unit_row<kEpi>(a, un, r) * (a.K / B) + k0 / B + cw * 4;
-          cp_async4(st_base + kScalesOff + r * kScaleRow + cw * 4, src);
+        if (kFmt != FP4_CB4) {
+          for (int w = lane; w < kRows * words; w += 32) {
+            const int r = w / words, cw = w - r * words;
+            const uint8_t* src = a.scales + unit_row<kEpi>(a, un, r) * (a.K / B) + k0 / B + cw * 4;
+            cp_async4(st_base + kScalesOff + r * kScaleRow + cw * 4, src);
+          }
+          cp_async_arrive(bar_full + 8 * s);
         }
-        cp_async_arrive(bar_full + 8 * s);
         __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         __syncwarp();
+        if (kFmt == FP4_CB4)
+          for (int r = lane; r < kRows; r += 32)
+            bulk_g2s(st_base + kScalesOff + r * kScaleRow, a.scales + unit_row<kEpi>(a, un, r) * (a.K / 4) + k0 / 4,
+                     static_cast<uint32_t>(kScaleRow), bar_full + 8 * s);
         for (int q = lane; q < 2 * ncb; q += 32) {
           const int rb = q & 1, cb = q >> 1;
           tma_load_2d(st_base + (cb * kRows + rb * 32) * 128, &tmap, k0 / 2 + cb * 128,
@@ -334,7 +376,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t c_xo[kNq];
 #pragma unroll
   for (int jj = 0; jj < kNq; ++jj) c_xo[jj] = static_cast<uint32_t>((((jbase & 7) + jj) ^ g) << 4);
-  const uint32_t s_off = kScalesOff + rbase * kScaleRow + (kFmt == FP4_MXFP4 ? jbase : 2 * jbase);
+  const uint32_t s_off = kScalesOff + rbase * kScaleRow +
+                         (kFmt == FP4_MXFP4 ? jbase : (kFmt == FP4_NVFP4 ? 2 * jbase : (jbase >> 2) * 32));
   const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
   int it = 0;
   while (true) {
@@ -360,10 +403,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint8_t* stp = smem + s * L.stage_bytes;
       // scale bytes of this warp's regions, one load per row
       uint32_t sb[4][(kFmt == FP4_MXFP4) ? 1 : 2];
+      // CB4: byte tables of the 16 fp16 entries of each of the warp's rows (one group)
+      uint32_t tlo[4][4], thi[4][4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const uint8_t* sp = stp + s_off + m * 8 * kScaleRow;
-        if (kFmt == FP4_MXFP4) {
+        if (kFmt == FP4_CB4) {
+          const uint4 c0 = *reinterpret_cast<const uint4*>(sp);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(sp + 16);
+          const uint32_t e[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            tlo[m][q] = __byte_perm(e[2 * q], e[2 * q + 1], 0x6420);
+            thi[m][q] = __byte_perm(e[2 * q], e[2 * q + 1], 0x7531);
+          }
+          sb[m][0] = 0u;
+        } else if (kFmt == FP4_MXFP4) {
           static_assert(kFmt != FP4_MXFP4 || kNq <= 4, "scale word");
           sb[m][0] = (kNq == 4) ? *reinterpret_cast<const uint32_t*>(sp) : *reinterpret_cast<const uint16_t*>(sp);
         } else if (kNq == 4) {
@@ -382,10 +437,21 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(cp + m * 8 * 128);
         uint32_t p[4][4];
+        if (kFmt == FP4_CB4) {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) e2m1x8_to_f16x8(w[m], p[m][0], p[m][1], p[m][2], p[m][3]);
+          for (int m = 0; m < 4; ++m) cb4_lookup8(w[m], tlo[m], thi[m], p[m]);
+        } else {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) e2m1x8_to_f16x8(w[m], p[m][0], p[m][1], p[m][2], p[m][3]);
+        }
         const uint4 xq = *reinterpret_cast<const uint4*>(stp + x_off + jj * 64);
-        if (kFmt == FP4_NVFP4) {
+        if (kFmt == FP4_CB4) {
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_16816(acc[mt], p[2 * mt][0], p[2 * mt + 1][0], p[2 * mt][1], p[2 * mt + 1][1], xq.x, xq.y);
+            mma_16816(acc[mt], p[2 * mt][2], p[2 * mt + 1][2], p[2 * mt][3], p[2 * mt + 1][3], xq.z, xq.w);
+          }
+        } else if (kFmt == FP4_NVFP4) {
           // this thread's 8 K positions lie in block 2j + (t >> 1): byte 2 jj + (t >> 1) of the row's run
           const int bsel = 2 * jj + (t >> 1);
           uint32_t b4[4];
@@ -446,13 +512,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
     // ---- fused epilogue ----
     const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e] : 1.0f;
+    // CB4 sparse term of row r against an activation row (same scaling as the MMA input)
+    auto sparse = [&](int r, const __half* xrow) -> float {
+      if (kFmt != FP4_CB4 || a.sp_rowptr == nullptr) return 0.f;
+      const int64_t R = unit_row<kEpi>(a, un, r);
+      float acc_s = 0.f;
+      for (int j = a.sp_rowptr[R]; j < a.sp_rowptr[R + 1]; ++j)
+        acc_s = fmaf(__half2float(__ushort_as_half(a.sp_val[j])), __half2float(xrow[a.sp_col[j]]), acc_s);
+      return acc_s;
+    };
     if (kEpi == kEpiSwiglu) {
       for (int idx = threadIdx.x; idx < 32 * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 31, i = idx >> 5;
         const int tok = perm_at(un.slot0 + i) / a.topk;
         const float sc = ldexpf(ts, a.sexp[tok]);
-        const float gv = fminf(val(r, i) * sc, a.limit);
-        const float uv = fminf(fmaxf(val(32 + r, i) * sc, -a.limit), a.limit);
+        const __half* xrow = a.x16 + static_cast<int64_t>(tok) * a.K;
+        const float gv = fminf((val(r, i) + sparse(r, xrow)) * sc, a.limit);
+        const float uv = fminf(fmaxf((val(32 + r, i) + sparse(32 + r, xrow)) * sc, -a.limit), a.limit);
         const float hv = gv / (1.0f + expf(-gv)) * uv;
         a.h_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * 32 + r] = __float2half_rn(hv);
       }
@@ -460,7 +536,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
         const float wgt = a.gw[perm_at(un.slot0 + i)];
-        a.o_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] = val(r, i) * ts * wgt;
+        const float v = val(r, i) + sparse(r, a.x16 + static_cast<int64_t>(un.slot0 + i) * a.K);
+        a.o_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] = v * ts * wgt;
       }
     } else {
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
@@ -477,11 +554,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 Layout make_layout(int fmt, int K, int E, int P) {
   Layout L{};
   const int B = (fmt == FP4_MXFP4) ? 32 : 16;
-  const int kc = (K % 512 == 0) ? 512 : ((K % 256 == 0) ? 256 : 0);
+  // CB4 stages carry 4 codebook bytes per 16 indices: the smaller stage keeps 5 in flight
+  const int kc = (fmt != FP4_CB4 && K % 512 == 0) ? 512 : ((K % 256 == 0) ? 256 : 0);
   if (kc == 0) return L;
   L.kc = kc;
   L.nchunks = K / kc;
-  L.scale_row = kc / B;
+  L.scale_row = (fmt == FP4_CB4) ? kc / 4 : kc / B;
   L.codes_off = 0;
   L.scales_off = kRows * kc / 2;
   L.x_off = L.scales_off + kRows * L.scale_row;
@@ -520,7 +598,9 @@ fp4_status launch_kc(const DecodeArgs& a, const Layout& L, const CUtensorMap& ma
 template <int kFmt, int kEpi, int kMode>
 fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
                       bool pdl) {
-  if (L.kc == 512) return launch_kc<kFmt, kEpi, kMode, 512>(a, L, map, grid, st, pdl);
+  if constexpr (kFmt != FP4_CB4) {
+    if (L.kc == 512) return launch_kc<kFmt, kEpi, kMode, 512>(a, L, map, grid, st, pdl);
+  }
   return launch_kc<kFmt, kEpi, kMode, 256>(a, L, map, grid, st, pdl);
 }
 
@@ -546,6 +626,7 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
                           static_cast<uint64_t>(a.K / 2), 128, 32, CU_TENSOR_MAP_SWIZZLE_128B));
   int grid = 2 * num_sms();
   if (a.mode == kModeStatic) grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok));
+  if (a.fmt == FP4_CB4) return dispatch<FP4_CB4>(a, L, map, grid, st, pdl);
   return (a.fmt == FP4_NVFP4) ? dispatch<FP4_NVFP4>(a, L, map, grid, st, pdl)
                               : dispatch<FP4_MXFP4>(a, L, map, grid, st, pdl);
 }

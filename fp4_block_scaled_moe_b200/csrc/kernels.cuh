@@ -64,11 +64,14 @@ constexpr int kRouteMaxPairs = 1024;   // kModeRoute limits (shared-memory routi
 constexpr int kRouteMaxExperts = 512;
 
 struct DecodeArgs {
-  int fmt;                       // FP4_MXFP4 / FP4_NVFP4
+  int fmt;                       // FP4_MXFP4 / FP4_NVFP4 / FP4_CB4
   int epi;                       // DecodeEpi
   int mode;                      // DecodeMode
-  const uint8_t* codes;          // [rows_total, K/2]
-  const uint8_t* scales;         // [rows_total, K/B]
+  const uint8_t* codes;          // [rows_total, K/2] (CB4: 4-bit codebook indices)
+  const uint8_t* scales;         // [rows_total, K/B] (CB4: fp16 codebooks [rows_total, K/128, 16])
+  const int32_t* sp_rowptr;      // CB4 sparse term: CSR over rows_total rows (or null)
+  const int32_t* sp_col;
+  const uint16_t* sp_val;        // fp16 bits
   const float* tscale;           // [E] (NVFP4) or null
   int64_t rows_total;
   int K;

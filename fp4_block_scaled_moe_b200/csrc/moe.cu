@@ -60,9 +60,7 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
 
 fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (w == nullptr) return FP4_ERR_INVALID_ARG;
-  if (w->fmt != FP4_MXFP4 && w->fmt != FP4_NVFP4) {
-    return (w->fmt == FP4_CB4) ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
-  }
+  if (w->fmt != FP4_MXFP4 && w->fmt != FP4_NVFP4 && w->fmt != FP4_CB4) return FP4_ERR_INVALID_ARG;
   int64_t n;
   FP4_TRY(checked_count({w->num_experts, w->hidden, w->inter, T}, &n));
   if (k <= 0) return FP4_ERR_EMPTY_SHAPE;
@@ -75,10 +73,19 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (!mul_ok(P, H * 4, &tmp) || !mul_ok(static_cast<int64_t>(T) * E, 4, &tmp)) return FP4_ERR_SHAPE_OVERFLOW;
   if (E * 2 * I >= (int64_t(1) << 31) || E * H >= (int64_t(1) << 31)) return FP4_ERR_SHAPE_OVERFLOW;
   if (k > E || k > 32 || E > 1024) return FP4_ERR_INVALID_ARG;
-  const int B = (w->fmt == FP4_MXFP4) ? 32 : 16;
+  const int B = (w->fmt == FP4_MXFP4) ? 32 : (w->fmt == FP4_NVFP4 ? 16 : 128);
   if (H % B != 0 || I % B != 0) return FP4_ERR_ALIGNMENT;
   if (H % 256 != 0 || I % 256 != 0) return FP4_ERR_UNSUPPORTED;
   if (!(w->swiglu_limit > 0.f) || !(w->swiglu_limit <= 128.f)) return FP4_ERR_INVALID_ARG;
+  if (w->fmt == FP4_CB4) {
+    if (!w->gu_codes || !w->gu_cb || !w->dn_codes || !w->dn_cb || !w->gu_rowptr || !w->dn_rowptr)
+      return FP4_ERR_INVALID_ARG;
+    if (!aligned16(w->gu_codes) || !aligned16(w->gu_cb) || !aligned16(w->dn_codes) || !aligned16(w->dn_cb))
+      return FP4_ERR_ALIGNMENT;
+    if (w->kernel_variant == kVarTensor) return FP4_ERR_UNSUPPORTED;
+    if (w->kernel_variant < 0 || w->kernel_variant > 2) return FP4_ERR_INVALID_ARG;
+    return FP4_OK;
+  }
   if (!w->gu_codes || !w->gu_scales || !w->dn_codes || !w->dn_scales) return FP4_ERR_INVALID_ARG;
   if (w->fmt == FP4_NVFP4 && (!w->gu_tscale || !w->dn_tscale)) return FP4_ERR_INVALID_ARG;
   if (w->kernel_variant < 0 || w->kernel_variant > 2) return FP4_ERR_INVALID_ARG;
@@ -195,8 +202,13 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   g.epi = kEpiSwiglu;
   g.mode = fused ? kModeRoute : kModeList;
   g.codes = w->gu_codes;
-  g.scales = w->gu_scales;
+  g.scales = (w->fmt == FP4_CB4) ? reinterpret_cast<const uint8_t*>(w->gu_cb) : w->gu_scales;
   g.tscale = w->gu_tscale;
+  if (w->fmt == FP4_CB4) {
+    g.sp_rowptr = w->gu_rowptr;
+    g.sp_col = w->gu_col;
+    g.sp_val = w->gu_val;
+  }
   g.rows_total = static_cast<int64_t>(E) * 2 * I;
   g.K = H;
   g.rows_per_expert = 2 * I;
@@ -225,8 +237,13 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   d.epi = kEpiDown;
   d.mode = kModeList;
   d.codes = w->dn_codes;
-  d.scales = w->dn_scales;
+  d.scales = (w->fmt == FP4_CB4) ? reinterpret_cast<const uint8_t*>(w->dn_cb) : w->dn_scales;
   d.tscale = w->dn_tscale;
+  if (w->fmt == FP4_CB4) {
+    d.sp_rowptr = w->dn_rowptr;
+    d.sp_col = w->dn_col;
+    d.sp_val = w->dn_val;
+  }
   d.rows_total = static_cast<int64_t>(E) * H;
   d.K = I;
   d.rows_per_expert = H;

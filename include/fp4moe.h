@@ -104,6 +104,34 @@ fp4_status fp4_unpack(fp4_format fmt, const uint8_t* codes, const uint8_t* scale
                       fp4_dtype out_dtype, void* stream);
 
 /*
+ * CB4 packing: a 16-entry fp16 codebook per 128-weight group of each row plus a sparse
+ * fp16 outlier term ("XFP：质量地板驱动的自适应码本量化", sections 离群值提取, Lloyd 迭代
+ * and the V2 dense + sparse decomposition; 4-bit indices as in 子字节打包).
+ * w [rows, k] float32 or bf16 (device), k % 128 == 0, rows * k < 2^31.  An outlier is
+ * a weight with |w - mu| > threshold (float64 comparison).
+ *   fp4_cb4_row_ptr: row_ptr [rows + 1] int32 (device) = exclusive scan of the outlier
+ *     counts per row; row_ptr[rows] = nnz.  Call it first to size col and val.
+ *   fp4_pack_cb4 (row_ptr from the first call): idx [rows, k/2] (even position in the low
+ *     nibble), cb [rows, k/128, 16] fp16 bits, col [nnz] int32 (column within the row,
+ *     ascending), val [nnz] fp16 bits.
+ * Per group: outliers are replaced by mu; the entries start at the sorted values at
+ * positions 8i + 4 (i = 0..15, the (i + 0.5)/16 quantiles); 20 Lloyd rounds assign each
+ * weight to its nearest entry (ties to the lower index) and set each entry to the mean
+ * of its members (summed in ascending position, float64; an empty entry is kept); the
+ * entries are rounded to fp16 (nearest even) and every weight is assigned once more to
+ * the nearest fp16 entry.  val = fp16(w - entry(idx)) at each outlier, so the dense
+ * term plus the sparse term approximates w.  Deterministic.  col and val may be NULL
+ * only when nnz == 0.  Errors: EMPTY_SHAPE, SHAPE_OVERFLOW, ALIGNMENT (k % 128, w, idx,
+ * cb not 16-byte aligned), INVALID_ARG (threshold negative or not finite, mu not
+ * finite, NULL pointers).
+ */
+fp4_status fp4_cb4_row_ptr(const void* w, fp4_dtype w_dtype, int64_t rows, int64_t k, double threshold,
+                           double mu, int32_t* row_ptr, void* stream);
+fp4_status fp4_pack_cb4(const void* w, fp4_dtype w_dtype, int64_t rows, int64_t k, double threshold, double mu,
+                        const int32_t* row_ptr, uint8_t* idx, uint16_t* cb, int32_t* col, uint16_t* val,
+                        void* stream);
+
+/*
  * moe_route: router of the MoE layer ("The gate that missed by 0.0202 pp", section
  * "A file is a census; a decode step is a sample": each token reads k of E experts).
  *   logits[t, e] = sum_h x[t, h] * router_w[e, h] + router_bias[e]   (float32 accumulate)

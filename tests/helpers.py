@@ -53,11 +53,13 @@ class LazyOracleBank:
         self._M = M
 
     def packed(self, which, e):
-        from oracle import formats as F
+        from oracle import codebook as CB, formats as F
         key = (which, e)
         if key not in self._cache:
             w = expert_host(self.cfg, which, e)
-            if self.cfg.fmt == "mxfp4":
+            if self.cfg.fmt == "cb4":
+                self._cache[key] = CB.cb4_fit(w, self.cfg.cb4_threshold_sigma * self.cfg.sigma)
+            elif self.cfg.fmt == "mxfp4":
                 self._cache[key] = F.mxfp4_quantize(w) + (None,)
             else:
                 c, s, t = F.nvfp4_quantize(w[None])
@@ -65,7 +67,12 @@ class LazyOracleBank:
         return self._cache[key]
 
     def dequant(self, which, e):
-        from oracle import formats as F
+        from oracle import codebook as CB, formats as F
+        if self.cfg.fmt == "cb4":
+            fit = self.packed(which, e)
+            n, k2 = fit["idx"].shape
+            return CB.cb4_dense(fit["idx"], fit["cb_val"]) + CB.cb4_sparse(fit["row_ptr"], fit["col"], fit["val"],
+                                                                           n, 2 * k2)
         c, s, t = self.packed(which, e)
         if self.cfg.fmt == "mxfp4":
             return F.mxfp4_dequantize(c, s)
@@ -78,11 +85,32 @@ class LazyOracleBank:
         return h @ self.dequant("dn", e).T
 
 
+def device_weights_cb4(cfg, device="cuda"):
+    """CB4 weights drawn on the device and packed there with fp4_pack_cb4 over each fused
+    expert matrix ([E * rows, K]; one CSR per matrix)."""
+    import torch
+    from fp4_block_scaled_moe_b200 import MoEWeights, fp4_pack_cb4
+    from synth import device as SD
+    out = {}
+    for which, tid, rows, K in (("gu", C.TID_GATE_UP, 2 * cfg.I, cfg.H), ("dn", C.TID_DOWN, cfg.H, cfg.I)):
+        w = torch.empty((cfg.E * rows, K), dtype=torch.float32, device=device)
+        SD.expert_weights_into(w, cfg.seed, tid, start_row=0, sigma=cfg.sigma, outliers=cfg.outliers)
+        out[which] = fp4_pack_cb4(w, cfg.cb4_threshold_sigma * cfg.sigma)
+        del w
+    gu, dn = out["gu"], out["dn"]
+    return MoEWeights(cfg.fmt, cfg.E, cfg.H, cfg.I, gu["idx"].view(cfg.E, 2 * cfg.I, cfg.H // 2), None,
+                      dn["idx"].view(cfg.E, cfg.H, cfg.I // 2), None, None, None, cfg.swiglu_limit,
+                      gu_cb=gu["cb"], gu_rowptr=gu["row_ptr"], gu_col=gu["col"], gu_val=gu["val"],
+                      dn_cb=dn["cb"], dn_rowptr=dn["row_ptr"], dn_col=dn["col"], dn_val=dn["val"])
+
+
 def device_weights(cfg, device="cuda", chunk_elems=1 << 28):
     """Draw every expert's weights on the device and pack them there with fp4_pack."""
     import torch
     from fp4_block_scaled_moe_b200 import MoEWeights, fp4_pack
     from synth import device as SD
+    if cfg.fmt == "cb4":
+        return device_weights_cb4(cfg, device)
     B = 32 if cfg.fmt == "mxfp4" else 16
     out = {}
     for which, tid, rows, K in (("gu", C.TID_GATE_UP, 2 * cfg.I, cfg.H), ("dn", C.TID_DOWN, cfg.H, cfg.I)):

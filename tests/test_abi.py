@@ -82,7 +82,11 @@ def test_forward_named_refusals():
     assert fwd(_weights(lim=float("inf"))) == 1
     assert fwd(_weights(lim=-1.0)) == 1
     assert fwd(_weights(), k=9) == 1
-    assert fwd(_weights(fmt=L.FP4_CB4)) == 5
+    assert fwd(_weights(fmt=L.FP4_CB4)) == 1           # CB4 without codebooks / CSR
+    cb = _weights(fmt=L.FP4_CB4)
+    cb.gu_cb = cb.dn_cb = cb.gu_rowptr = cb.dn_rowptr = 0x10000
+    cb.kernel_variant = 2
+    assert fwd(cb) == 5                                 # CB4 runs on the CUDA-core kernels only
     assert fwd(_weights(E=1 << 20, H=1 << 16, I=1 << 16)) == 3
     assert fwd(_weights(), ws=None) == 6
     bad = _weights()

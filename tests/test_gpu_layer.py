@@ -62,10 +62,16 @@ def _moe_case(cfg, tokens=None, variant=0):
     return check_tolerance(got, ref, mask_rows=ok)
 
 
-@pytest.mark.parametrize("cfg", [C.small(C.MOE_C2), C.small(C.MOE_C3), C.small(C.MOE_C4)],
-                         ids=["c2_small", "c3_small", "c4_small_prefill_shape"])
+@pytest.mark.parametrize("cfg", [C.small(C.MOE_C2), C.small(C.MOE_C3), C.small(C.MOE_C4), C.small(C.MOE_C5)],
+                         ids=["c2_small", "c3_small", "c4_small_prefill_shape", "c5_small_cb4"])
 def test_moe_small(cfg):
     _moe_case(cfg)
+
+
+def test_moe_c5_cb4_full_sampled_tokens():
+    """The CB4 decode layer at full size (64 experts, hidden 2048, intermediate 768,
+    top-8, 16 tokens; codebooks per 128 weights plus the CSR outlier term)."""
+    _moe_case(C.MOE_C5, tokens=[9])
 
 
 def test_moe_c2_full_sampled_tokens():
