@@ -8,6 +8,7 @@ from .api import (  # noqa: F401
     alloc_workspace,
     fp4_launch_count,
     fp4_linear,
+    fp4_mma_scales,
     fp4_pack,
     fp4_pack_cb4,
     fp4_unpack,
@@ -17,6 +18,7 @@ from .api import (  # noqa: F401
     moe_fp4_forward_noalloc,
     moe_fp4_workspace_size,
     moe_route,
+    prepare_mma_scales,
 )
 
 __version__ = "0.1.0"

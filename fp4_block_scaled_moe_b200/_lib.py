@@ -35,6 +35,7 @@ class MoEWeightsC(ctypes.Structure):
         ("gu_cb", _vp), ("gu_rowptr", _vp), ("gu_col", _vp), ("gu_val", _vp),
         ("dn_cb", _vp), ("dn_rowptr", _vp), ("dn_col", _vp), ("dn_val", _vp),
         ("kernel_variant", _i32),
+        ("gu_mma_scales", _vp), ("dn_mma_scales", _vp),
     ]
 
 
@@ -54,6 +55,7 @@ SIGNATURES = {
     "fp4_version": (ctypes.c_char_p, []),
     "fp4_launch_count": (ctypes.c_ulonglong, []),
     "fp4_pack": (_cint, [_cint, _vp, _cint, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "fp4_mma_scales": (_cint, [_vp, _i64, _i64, _vp, _vp]),
     "fp4_cb4_row_ptr": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp]),
     "fp4_pack_cb4": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp, _vp, _vp, _vp,
                              _vp]),

@@ -58,6 +58,23 @@ def fp4_pack(w: torch.Tensor, fmt="mxfp4"):
     return codes, scales, ts
 
 
+def fp4_mma_scales(scales: torch.Tensor) -> torch.Tensor:
+    """MXFP4 scales [..., rows, k/32] re-laid as tensor-core scale atoms (flat uint8)."""
+    _need(scales, "scales", torch.uint8)
+    k = scales.shape[-1] * 32
+    rows = scales.numel() // scales.shape[-1]
+    out = torch.empty(scales.numel(), dtype=torch.uint8, device=scales.device)
+    L.check("fp4_mma_scales", L.load().fp4_mma_scales(_ptr(scales), rows, k, _ptr(out), _stream(scales.device)))
+    return out
+
+
+def prepare_mma_scales(weights: "MoEWeights") -> "MoEWeights":
+    """Attach re-laid gate_up / down scales to MXFP4 weights for the tensor-core kernels."""
+    weights.gu_mma_scales = fp4_mma_scales(weights.gu_scales)
+    weights.dn_mma_scales = fp4_mma_scales(weights.dn_scales)
+    return weights
+
+
 def fp4_pack_cb4(w: torch.Tensor, threshold: float, mu: float = 0.0):
     """CB4 pack of w [rows, k] (float32 or bf16): returns dict(idx, cb, row_ptr, col, val)
     (see fp4_cb4_row_ptr / fp4_pack_cb4 in include/fp4moe.h)."""
@@ -153,6 +170,9 @@ class MoEWeights:
     dn_val: torch.Tensor | None = None
     # expert-GEMM kernels: 0 chosen per call, 1 CUDA-core GEMV, 2 tensor-core (MXFP4)
     kernel_variant: int = 0
+    # tensor-core kernels: scales re-laid by fp4_mma_scales (else re-laid every call)
+    gu_mma_scales: torch.Tensor | None = None
+    dn_mma_scales: torch.Tensor | None = None
 
     def c_struct(self):
         s = L.MoEWeightsC()
@@ -161,7 +181,8 @@ class MoEWeights:
         s.swiglu_limit = self.swiglu_limit
         s.kernel_variant = self.kernel_variant
         for name in ("gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales", "dn_tscale", "gu_cb",
-                     "gu_rowptr", "gu_col", "gu_val", "dn_cb", "dn_rowptr", "dn_col", "dn_val"):
+                     "gu_rowptr", "gu_col", "gu_val", "dn_cb", "dn_rowptr", "dn_col", "dn_val", "gu_mma_scales",
+                     "dn_mma_scales"):
             t = getattr(self, name)
             setattr(s, name, None if t is None else t.data_ptr())
         return s

@@ -17,9 +17,9 @@
 //
 // Warp roles of one persistent CTA per SM:
 //   warp 0     producer: TMA of the two weight tiles (FP4 widened to 16-byte slots,
-//              128-byte swizzle) and of the activation-term tile; 4-byte async copies
-//              place the scale bytes in the 32-row x 16-byte atoms the TMEM scale copy
-//              reads.
+//              128-byte swizzle) and of the activation-term tile, and one bulk copy per
+//              scale atom (weights: re-laid once by fp4_mma_scales or per call into the
+//              workspace; activations: written as atoms by their producers).
 //   warp 1     MMA issuer and TMEM owner: per stage, scales -> TMEM, then 2 x 4 MMAs of
 //              K = 32 into one of two double-buffered accumulator pairs.
 //   warps 2-5  epilogue, one TMEM lane quadrant each: term pairs summed; gate_up applies
@@ -41,6 +41,7 @@ constexpr int kATile = 128 * 128;         // shared bytes of one 128-row FP4 til
 constexpr int kSfBytes = 3 * 512;         // scale atoms per stage: A0, A1, B
 constexpr int kSfCols = 16;               // TMEM columns per stage for scales (4 each)
 constexpr int kMaxTokCap = 56;            // tokens per unit: accumulators of 2 x 56 columns
+constexpr int kMaxExperts = 1024;
 
 struct BsLayout {
   int ntok_cap;      // tokens per work unit
@@ -53,7 +54,7 @@ struct BsLayout {
 };
 
 struct BsUnit {
-  int e, tile, slot0, ntok;
+  int e, tile, slot0, ntok, gid;    // gid: token group number across experts
 };
 
 __device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* off, const int* pre, int E,
@@ -72,17 +73,10 @@ __device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* o
   const int grp = local - un.tile * groups;
   un.slot0 = off[lo] + grp * cap;
   un.ntok = min(cap, n - grp * cap);
+  un.gid = pre[lo] / tiles + grp;
   return un;
 }
 
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-// Arrive on the mbarrier when this thread's earlier cp.async copies land (the pending
-// count is raised first, so the expected arrival count is unchanged).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 
 // byte offset of row r (0..127) in a scale atom: 32 rows x 16 bytes, row r at line r % 32,
 // word r / 32 (the four bytes of a word are the four 32-element blocks of one stage)
@@ -132,17 +126,51 @@ __device__ __forceinline__ void warp_split2(float v, uint32_t& q1, uint32_t& q2,
   s2 = static_cast<uint32_t>(e2 + 127);
 }
 
-// x [T][H] bf16 -> slot-ordered two-term MXFP8 rows: q [2P][H] E4M3, s [2P][H/32] UE8M0,
-// rows 2i, 2i + 1 for slot i (token perm[i] / k).  One thread per 32-element block.
+// x [T][H] bf16 -> slot-ordered two-term MXFP8 rows q [2P][H] E4M3 (rows 2i, 2i + 1 for
+// slot i = token perm[i] / k) and their UE8M0 scales as token-group atoms.  One thread
+// per 32-element block.
 __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict__ x,
-                                                      const int32_t* __restrict__ perm, int k, int P, int H,
-                                                      uint8_t* __restrict__ q, uint8_t* __restrict__ s) {
+                                                      const int32_t* __restrict__ perm,
+                                                      const int32_t* __restrict__ counts,
+                                                      const int32_t* __restrict__ offsets, int E, int k, int P,
+                                                      int H, int cap, uint8_t* __restrict__ q,
+                                                      uint8_t* __restrict__ atoms) {
+  __shared__ int off_s[kMaxExperts + 1], gpre_s[kMaxExperts + 1];
   pdl_wait();
-  const int nb = H / 32;
+  // group number of each expert's first group: exclusive scan of ceil(count / cap)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int sg = 0;
+    for (int e = e0; e < e1; ++e) sg += (counts[e] + cap - 1) / cap;
+    int ig = sg;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, ig, o);
+      if (lane >= o) ig += v;
+    }
+    int rg = ig - sg;
+    for (int e = e0; e < e1; ++e) {
+      gpre_s[e] = rg;
+      rg += (counts[e] + cap - 1) / cap;
+    }
+  }
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) off_s[e] = offsets[e];
+  __syncthreads();
+  const int nb = H / 32, kb128 = H / 128;
   const int64_t total = static_cast<int64_t>(P) * nb;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int slot = static_cast<int>(idx / nb), b = static_cast<int>(idx % nb);
+    int lo = 0, hi = E - 1;                    // expert of the slot: largest e with off[e] <= slot
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off_s[mid] <= slot) lo = mid; else hi = mid - 1;
+    }
+    const int local = slot - off_s[lo];
+    const int grp = local / cap, i = local - grp * cap;
+    const int64_t gid = gpre_s[lo] + grp;
     const int t = perm[slot] / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + 32 * b);
     float v[32];
@@ -151,35 +179,35 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
       const uint4 w = src[j];
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[8 * j + 2 * i] = __uint_as_float(ws[i] << 16);
-        v[8 * j + 2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+      for (int ii = 0; ii < 4; ++ii) {
+        v[8 * j + 2 * ii] = __uint_as_float(ws[ii] << 16);
+        v[8 * j + 2 * ii + 1] = __uint_as_float(ws[ii] & 0xFFFF0000u);
       }
     }
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int ii = 0; ii < 32; ++ii) amax = fmaxf(amax, fabsf(v[ii]));
     const int e1 = e4m3_block_exp(amax);
     const float inv1 = exp2i(-e1), up1 = exp2i(e1);
     uint32_t w1[8], w2[8];
     float ramax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int ii = 0; ii < 32; ++ii) {
       float b1;
-      const uint32_t c = e4m3_rn(v[i] * inv1, b1);
-      if ((i & 3) == 0) w1[i >> 2] = 0;
-      w1[i >> 2] |= c << (8 * (i & 3));
-      v[i] -= b1 * up1;
-      ramax = fmaxf(ramax, fabsf(v[i]));
+      const uint32_t c = e4m3_rn(v[ii] * inv1, b1);
+      if ((ii & 3) == 0) w1[ii >> 2] = 0;
+      w1[ii >> 2] |= c << (8 * (ii & 3));
+      v[ii] -= b1 * up1;
+      ramax = fmaxf(ramax, fabsf(v[ii]));
     }
     const int e2 = e4m3_block_exp(ramax);
     const float inv2 = exp2i(-e2);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int ii = 0; ii < 32; ++ii) {
       float b2;
-      const uint32_t c = e4m3_rn(v[i] * inv2, b2);
-      if ((i & 3) == 0) w2[i >> 2] = 0;
-      w2[i >> 2] |= c << (8 * (i & 3));
+      const uint32_t c = e4m3_rn(v[ii] * inv2, b2);
+      if ((ii & 3) == 0) w2[ii >> 2] = 0;
+      w2[ii >> 2] |= c << (8 * (ii & 3));
     }
     uint4* d1 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot)) * H + 32 * b);
     uint4* d2 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot) + 1) * H + 32 * b);
@@ -187,10 +215,24 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
     d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
     d2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
     d2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
-    s[(2 * static_cast<int64_t>(slot)) * nb + b] = static_cast<uint8_t>(e1 + 127);
-    s[(2 * static_cast<int64_t>(slot) + 1) * nb + b] = static_cast<uint8_t>(e2 + 127);
+    uint8_t* at = atoms + (gid * kb128 + (b >> 2)) * 512 + (b & 3);
+    at[sf_row_off(2 * i)] = static_cast<uint8_t>(e1 + 127);
+    at[sf_row_off(2 * i + 1)] = static_cast<uint8_t>(e2 + 127);
   }
   pdl_launch_dependents();
+}
+
+// Weight scales [rows][K/32] -> atoms: one thread moves the 4-byte word of one row and
+// one 128-K block.
+__global__ void __launch_bounds__(256) mma_scales_kernel(const uint8_t* __restrict__ scales, int64_t rows,
+                                                         int64_t K, uint8_t* __restrict__ atoms) {
+  const int64_t kb = K / 128, total = rows * kb;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / kb, c = idx % kb;
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(scales + r * (K / 32) + 4 * c);
+    *reinterpret_cast<uint32_t*>(atoms + ((r >> 7) * kb + c) * 512 + sf_row_off(static_cast<int>(r & 127))) = w;
+  }
 }
 
 template <int kEpi>
@@ -274,7 +316,6 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   __syncthreads();
   const int n_units = pre[E];
   const int nk = a.K / kKT;
-  const int ksf = a.K / 32;             // scale bytes per row
   const uint32_t stg = static_cast<uint32_t>(L.stage_bytes);
   const uint32_t b_off = 2 * kATile, sf_off = 2 * kATile + L.ncols * kKT;   // within a stage
 
@@ -298,10 +339,10 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const int64_t rbase = static_cast<int64_t>(un.e) * a.rows_per_expert;
       const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 128 : rbase + un.tile * 256;
       const int64_t y1 = (kEpi == kEpiSwiglu) ? y0 + a.inter : y0 + 128;
-      const int brow0 = 2 * un.slot0, nrows = 2 * un.ntok;
-      const uint8_t* sa0 = a.a_scales + y0 * ksf;
-      const uint8_t* sa1 = a.a_scales + y1 * ksf;
-      const uint8_t* sb = a.b_scales + static_cast<int64_t>(brow0) * ksf;
+      const int brow0 = 2 * un.slot0;
+      const uint8_t* sa0 = a.a_atoms + (y0 >> 7) * nk * 512;
+      const uint8_t* sa1 = a.a_atoms + (y1 >> 7) * nk * 512;
+      const uint8_t* sb = a.b_atoms + static_cast<int64_t>(un.gid) * nk * 512;
       for (int c = 0; c < nk; ++c, ++it) {
         const int s = it % S;
         if (it >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / S) & 1) ^ 1, a.status))) {
@@ -311,18 +352,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st = sbase + s * stg;
         const uint32_t sf = st + sf_off;
-        const int kb = c * (kKT / 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = lane + 32 * i;
-          cp_async4(sf + sf_row_off(r), sa0 + static_cast<int64_t>(r) * ksf + kb);
-          cp_async4(sf + 512 + sf_row_off(r), sa1 + static_cast<int64_t>(r) * ksf + kb);
-        }
-        for (int r = lane; r < nrows; r += 32) cp_async4(sf + 1024 + sf_row_off(r), sb + static_cast<int64_t>(r) * ksf + kb);
-        cp_async_mbar_arrive(bar_full + 8 * s);
-        __syncwarp();
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(2 * 128 * kKT / 2 + L.ncols * kKT));
+          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(2 * 128 * kKT / 2 + L.ncols * kKT + kSfBytes));
+          bulk_g2s(sf, sa0 + c * 512, 512, bar_full + 8 * s);
+          bulk_g2s(sf + 512, sa1 + c * 512, 512, bar_full + 8 * s);
+          bulk_g2s(sf + 1024, sb + c * 512, 512, bar_full + 8 * s);
           tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * s);
           tma_load_2d(st + kATile, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
           tma_load_2d(st + b_off, &tmB, c * kKT, brow0, bar_full + 8 * s);
@@ -370,7 +404,6 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         }
         tc::fence_after_sync();
         if (lane == 0) {
-          fence_proxy_async();    // scale bytes from cp.async, read next by the tensor-core copy
           const uint32_t st = sbase + s * stg;
           const uint32_t sf = st + sf_off;
           const uint32_t t0 = sf_t0 + s * kSfCols;
@@ -414,7 +447,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const int N = (2 * un.ntok + 15) & ~15;
       if (kEpi == kEpiSwiglu) {
         const int64_t col = static_cast<int64_t>(un.tile) * 128 + row;
-        const int64_t scol = col >> 5;
+        uint8_t* hat = a.h_atoms + (static_cast<int64_t>(un.gid) * (a.inter / 128) + un.tile) * 512 + q;
         for (int c0 = 0; c0 < N; c0 += 16) {
           uint32_t vg[16], vu[16];
           tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), vg);
@@ -433,8 +466,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
               a.hq[r0 * a.inter + col] = static_cast<uint8_t>(q1);
               a.hq[(r0 + 1) * a.inter + col] = static_cast<uint8_t>(q2);
               if (lane == 0) {
-                a.hs[r0 * (a.inter / 32) + scol] = static_cast<uint8_t>(s1);
-                a.hs[(r0 + 1) * (a.inter / 32) + scol] = static_cast<uint8_t>(s2);
+                hat[sf_row_off(2 * i)] = static_cast<uint8_t>(s1);
+                hat[sf_row_off(2 * i + 1)] = static_cast<uint8_t>(s2);
               }
             }
           }
@@ -514,11 +547,31 @@ bool bs_layout(int T, int E, BsLayout* L) {
 
 }  // namespace
 
-fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, int k, int P, int H, uint8_t* q, uint8_t* s,
-                          cudaStream_t st) {
+fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t* counts, const int32_t* offsets,
+                          int E, int k, int P, int H, int ntok_cap, uint8_t* q, uint8_t* atoms, cudaStream_t st) {
   const int64_t total = static_cast<int64_t>(P) * (H / 32);
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, num_sms() * 16)));
-  return launch_pdl(split_x_kernel, dim3(grid), dim3(256), 0, st, true, x, perm, k, P, H, q, s);
+  return launch_pdl(split_x_kernel, dim3(grid), dim3(256), 0, st, true, x, perm, counts, offsets, E, k, P, H,
+                    ntok_cap, q, atoms);
+}
+
+fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st) {
+  const int64_t total = rows * (K / 128);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, num_sms() * 16)));
+  mma_scales_kernel<<<grid, 256, 0, st>>>(scales, rows, K, atoms);
+  FP4_TRY_CUDA(cudaGetLastError());
+  note_launch();
+  return FP4_OK;
+}
+
+int bs_ntok_cap(int T, int E) {
+  BsLayout L;
+  return bs_layout(T, E, &L) ? L.ntok_cap : 0;
+}
+
+size_t bs_group_atom_bytes(int P, int E, int ntok_cap, int K) {
+  const size_t groups = static_cast<size_t>(P) / ntok_cap + E + 1;   // >= sum over experts of ceil(n_e / cap)
+  return groups * (K / 128) * 512;
 }
 
 bool bs_supported(int T, int E, int H, int I) {
@@ -528,7 +581,7 @@ bool bs_supported(int T, int E, int H, int I) {
 
 fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
   BsLayout L;
-  if (!bs_layout(T, a.E, &L)) return FP4_ERR_UNSUPPORTED;
+  if (!bs_layout(T, a.E, &L) || L.ntok_cap != a.ntok_cap) return FP4_ERR_UNSUPPORTED;
   CUtensorMap mA, mB;
   FP4_TRY(make_tmap_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.codes, static_cast<uint64_t>(a.K),
                        static_cast<uint64_t>(a.rows_total), static_cast<uint64_t>(a.K / 2), kKT, 128,

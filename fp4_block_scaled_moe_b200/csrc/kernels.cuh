@@ -106,22 +106,30 @@ __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __res
 
 
 // Block-scaled tensor-core expert GEMM (MXFP4 weights x two-term MXFP8 activations).
+// Scale atoms: 512 bytes holding the UE8M0 scales of 128 rows x 128 K (four 32-blocks):
+// row r, block b at byte (r % 32) * 16 + (r / 32) * 4 + b -- the layout the TMEM scale
+// copy (tcgen05.cp 32x128b, warpx4) reads.  Weights: atom (row block, K block) at
+// ((row / 128) * (K / 128) + k / 128) * 512.  Activation terms: one atom per (token
+// group, K block) at (group * (K / 128) + k / 128) * 512, rows 2i, 2i + 1 = the two
+// terms of the group's i-th slot; groups are the per-expert runs of ntok_cap slots,
+// numbered across experts in expert order.
 struct BsArgs {
   int epi;                        // kEpiSwiglu (gate_up + SwiGLU) or kEpiDown
   const uint8_t* codes;           // A: [rows_total][K/2] E2M1 pairs
-  const uint8_t* a_scales;        // A: [rows_total][K/32] UE8M0
+  const uint8_t* a_atoms;         // A: scale atoms of the weights
   int64_t rows_total;
   int K;
   int rows_per_expert;
   int inter;                      // I (gate rows, then up rows, per expert)
   int E;
   int P;                          // routed slots T*k
+  int ntok_cap;                   // slots per token group
   const int32_t* counts;
   const uint8_t* b_q;             // B: [2P][K] E4M3, rows 2i and 2i+1 = terms of slot i
-  const uint8_t* b_scales;        // B: [2P][K/32] UE8M0
+  const uint8_t* b_atoms;         // B: scale atoms per token group
   float limit;
   uint8_t* hq;                    // gate_up out: h terms [2P][I] E4M3
-  uint8_t* hs;                    //              [2P][I/32] UE8M0
+  uint8_t* h_atoms;               //              scale atoms per token group (K = I)
   const float* gw;                // down: gate weights by pair, perm: slot -> pair
   const int32_t* perm;
   float* o_out;                   // down out: [P][ldo] fp32, slot order
@@ -130,9 +138,14 @@ struct BsArgs {
   KernelSlot* slot;
   uint32_t* unit_next;
 };
+// slots per token group of the tensor-core kernels for T tokens (0 when unsupported)
+int bs_ntok_cap(int T, int E);
+// bytes of the activation scale atoms for P slots over E experts at this K
+size_t bs_group_atom_bytes(int P, int E, int ntok_cap, int K);
+fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st);
 bool bs_supported(int T, int E, int H, int I);
 fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st);
-fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, int k, int P, int H, uint8_t* q, uint8_t* s,
-                          cudaStream_t st);
+fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t* counts, const int32_t* offsets,
+                          int E, int k, int P, int H, int ntok_cap, uint8_t* q, uint8_t* atoms, cudaStream_t st);
 
 }  // namespace fp4

@@ -24,7 +24,7 @@ int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
 }
 
 struct MoeWs {
-  size_t status, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, h, o, xq, xs, hq, hs, total;
+  size_t status, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, h, o, xq, xs, hq, hs, agu, adn, total;
 };
 
 bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
@@ -49,11 +49,15 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   L->x16 = take(tensor ? 0 : sizeof(uint16_t) * T * H);
   L->h = take(tensor ? 0 : sizeof(uint16_t) * P * I);
   L->o = take(sizeof(float) * P * H);
-  // tensor-core variant: x and h as two MXFP8 terms per slot (rows 2i, 2i + 1)
+  // tensor-core variant: x and h as two MXFP8 terms per slot (rows 2i, 2i + 1), their
+  // scale atoms per token group, and the weights' scale atoms unless the caller has them
+  const int cap = tensor ? bs_ntok_cap(T, static_cast<int>(E)) : 1;
   L->xq = take(tensor ? 2 * P * H : 0);
-  L->xs = take(tensor ? 2 * P * (H / 32) : 0);
+  L->xs = take(tensor ? bs_group_atom_bytes(static_cast<int>(P), static_cast<int>(E), cap, static_cast<int>(H)) : 0);
   L->hq = take(tensor ? 2 * P * I : 0);
-  L->hs = take(tensor ? 2 * P * (I / 32) : 0);
+  L->hs = take(tensor ? bs_group_atom_bytes(static_cast<int>(P), static_cast<int>(E), cap, static_cast<int>(I)) : 0);
+  L->agu = take(tensor && w->gu_mma_scales == nullptr ? E * 2 * I * (H / 32) : 0);
+  L->adn = take(tensor && w->dn_mma_scales == nullptr ? E * H * (I / 32) : 0);
   L->total = off;
   return true;
 }
@@ -93,6 +97,7 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
     return FP4_ERR_UNSUPPORTED;
   if (!aligned16(w->gu_codes) || !aligned16(w->gu_scales) || !aligned16(w->dn_codes) || !aligned16(w->dn_scales))
     return FP4_ERR_ALIGNMENT;
+  if (!aligned16(w->gu_mma_scales) || !aligned16(w->dn_mma_scales)) return FP4_ERR_ALIGNMENT;
   return FP4_OK;
 }
 
@@ -148,11 +153,24 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     FP4_TRY(launch_route(ra, st));
     uint8_t* xq = ws + L.xq;
     uint8_t* xs = ws + L.xs;
-    FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, k, P, H, xq, xs, st));
+    const int cap = bs_ntok_cap(T, E);
+    const uint8_t* agu = w->gu_mma_scales;
+    const uint8_t* adn = w->dn_mma_scales;
+    if (agu == nullptr) {
+      FP4_TRY(launch_mma_scales(w->gu_scales, static_cast<int64_t>(E) * 2 * I, H, ws + L.agu, st));
+      agu = ws + L.agu;
+    }
+    if (adn == nullptr) {
+      FP4_TRY(launch_mma_scales(w->dn_scales, static_cast<int64_t>(E) * H, I, ws + L.adn, st));
+      adn = ws + L.adn;
+    }
+    FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, ra.counts, ra.offsets, E, k, P, H, cap, xq,
+                           xs, st));
     BsArgs g{};
     g.epi = kEpiSwiglu;
     g.codes = w->gu_codes;
-    g.a_scales = w->gu_scales;
+    g.a_atoms = agu;
+    g.ntok_cap = cap;
     g.rows_total = static_cast<int64_t>(E) * 2 * I;
     g.K = H;
     g.rows_per_expert = 2 * I;
@@ -161,10 +179,10 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     g.P = P;
     g.counts = ra.counts;
     g.b_q = xq;
-    g.b_scales = xs;
+    g.b_atoms = xs;
     g.limit = w->swiglu_limit;
     g.hq = ws + L.hq;
-    g.hs = ws + L.hs;
+    g.h_atoms = ws + L.hs;
     g.status = &ra.ctrl->status;
     g.slot = &ra.ctrl->slot[0];
     g.unit_next = &ra.ctrl->unit_next[0];
@@ -172,12 +190,12 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     BsArgs d = g;
     d.epi = kEpiDown;
     d.codes = w->dn_codes;
-    d.a_scales = w->dn_scales;
+    d.a_atoms = adn;
     d.rows_total = static_cast<int64_t>(E) * H;
     d.K = I;
     d.rows_per_expert = H;
     d.b_q = g.hq;
-    d.b_scales = g.hs;
+    d.b_atoms = g.h_atoms;
     d.gw = ra.gw;
     d.perm = ra.perm;
     d.o_out = reinterpret_cast<float*>(ws + L.o);

