@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default=C.MOE_C2.name, choices=sorted(C.FULL))
+    ap.add_argument("--config", default=C.MOE_C2.name, choices=sorted(C.FULL) + sorted(C.PROFILE))
     ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2],
                     help="expert kernels: 0 chosen by the library, 1 CUDA-core GEMV, 2 tensor cores (MXFP4)")
     ap.add_argument("--no-clocks", action="store_true")
@@ -338,6 +338,16 @@ def oracle_sample(cfg, n_tokens):
     return run, work_per_step(cfg, counts, tokens=n_tokens, extra=extra)[0]
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel from one ncu capture of the
+# current build (profiles/): the decode layer's gate_up decode_kernel, and the prefill
+# gate_up bs_moe_kernel captured at a quarter of the experts and tokens and scaled by the
+# four times as many work units of the full layer.  None when no capture matches.
+NCU_TRAFFIC = {
+    ("moe_mxfp4_decode_e64_h2048_i768_k8_t16", "decode_kernel<gate_up+swiglu>"): 101_306_368,
+    ("moe_mxfp4_prefill_e256_h6144_i2048_k8_t8192", "bs_moe_kernel<gate_up+swiglu>"): 4 * 1_137_554_392,
+}
+
+
 def roofline(cfg, r, hbm_peak, peaks, tensor=False):
     """Dominant kernel: gate_up with the fused SwiGLU, timed per launch on the device.
     Prefill: algorithmic flops per launch 4 T k H I against the measured bf16 peak (the
@@ -352,7 +362,8 @@ def roofline(cfg, r, hbm_peak, peaks, tensor=False):
         ach = flops / (ms * 1e-3) / 1e12 if ms > 0 else None
         peak = peaks.get("bf16_tflops", 1590.0)
         return {"kernel": "bs_moe_kernel<gate_up+swiglu>", "bound": "tensor", "achieved": ach, "peak": peak,
-                "unit": "TFLOP/s", "frac": (ach / peak) if ach else None, "traffic": None,
+                "unit": "TFLOP/s", "frac": (ach / peak) if ach else None,
+                "traffic": NCU_TRAFFIC.get((cfg.name, "bs_moe_kernel<gate_up+swiglu>")),
                 "peak_source": ("MEASURED_PEAKS.json bf16_tflops, burst (of measured)" if "bf16_tflops" in peaks
                                 else "fallback 1590 TFLOP/s bf16 (of fallback)"),
                 "frac_of_sustained": (ach / peaks["bf16_tflops_sustained"]) if ach and "bf16_tflops_sustained" in peaks
@@ -366,8 +377,9 @@ def roofline(cfg, r, hbm_peak, peaks, tensor=False):
     if r.get("extra_gu") is not None:
         alg += int(np.sum(r["extra_gu"][r["counts"] > 0]))
     ach = alg / (ms * 1e-3) / 1e9 if ms > 0 else None
-    return {"kernel": "bs_moe_kernel<gate_up+swiglu>" if tensor else "decode_kernel<gate_up+swiglu>", "bound": "hbm", "achieved": ach, "peak": hbm_peak,
-            "unit": "GB/s", "frac": (ach / hbm_peak) if ach else None, "traffic": None,
+    kname = "bs_moe_kernel<gate_up+swiglu>" if tensor else "decode_kernel<gate_up+swiglu>"
+    return {"kernel": kname, "bound": "hbm", "achieved": ach, "peak": hbm_peak,
+            "unit": "GB/s", "frac": (ach / hbm_peak) if ach else None, "traffic": NCU_TRAFFIC.get((cfg.name, kname)),
             "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if "hbm_gbs" in peaks else "fallback",
             "bytes_per_launch": int(alg), "ms_per_launch": ms, "down_ms_per_launch": r["kern_ms"]["down"],
             "timer": "device globaltimer per launch, accumulated in the workspace over the timed steps"}
@@ -405,7 +417,7 @@ def blas_threads():
 
 def main():
     args = parse()
-    cfg = C.FULL[args.config]
+    cfg = C.FULL.get(args.config) or C.PROFILE[args.config]
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     metric = "FP4 MoE layer: decode HBM GB/s (% of peak); prefill TFLOP/s; tokens/s"

@@ -64,6 +64,11 @@ MOE_C5 = MoEConfig("moe_cb4_decode_e64_h2048_i768_k8_t16", "cb4", T=16, E=64, H=
                    outliers=(0.00394, 6.0, 49.0))
 
 FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5)}
+# The prefill layer at a quarter of the experts and tokens (same per-expert load, same
+# tile shapes; 1.3 GB of weights): the size used for full hardware-counter captures.
+MOE_C4_PROFILE = MoEConfig("moe_mxfp4_prefill_e64_h6144_i2048_k8_t2048", "mxfp4", T=2048, E=64, H=6144,
+                           I=2048, k=8)
+PROFILE = {MOE_C4_PROFILE.name: MOE_C4_PROFILE}
 
 
 def small(cfg):
