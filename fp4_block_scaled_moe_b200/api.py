@@ -58,19 +58,20 @@ def fp4_pack(w: torch.Tensor, fmt="mxfp4"):
     return codes, scales, ts
 
 
-def fp4_mma_scales(scales: torch.Tensor) -> torch.Tensor:
-    """MXFP4 scales [..., rows, k/32] re-laid as tensor-core scale atoms (flat uint8)."""
+def fp4_mma_scales(scales: torch.Tensor, pair: int = 0) -> torch.Tensor:
+    """MXFP4 scales [..., rows, k/32] re-laid as tensor-core scale atoms (flat uint8);
+    pair = I for gate_up weights (tiles of 64 gate + 64 up rows), 0 for down weights."""
     _need(scales, "scales", torch.uint8)
     k = scales.shape[-1] * 32
     rows = scales.numel() // scales.shape[-1]
     out = torch.empty(scales.numel(), dtype=torch.uint8, device=scales.device)
-    L.check("fp4_mma_scales", L.load().fp4_mma_scales(_ptr(scales), rows, k, _ptr(out), _stream(scales.device)))
+    L.check("fp4_mma_scales", L.load().fp4_mma_scales(_ptr(scales), rows, k, pair, _ptr(out), _stream(scales.device)))
     return out
 
 
 def prepare_mma_scales(weights: "MoEWeights") -> "MoEWeights":
     """Attach re-laid gate_up / down scales to MXFP4 weights for the tensor-core kernels."""
-    weights.gu_mma_scales = fp4_mma_scales(weights.gu_scales)
+    weights.gu_mma_scales = fp4_mma_scales(weights.gu_scales, pair=weights.I)
     weights.dn_mma_scales = fp4_mma_scales(weights.dn_scales)
     return weights
 

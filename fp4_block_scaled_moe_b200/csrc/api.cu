@@ -140,11 +140,15 @@ extern "C" fp4_status fp4_workspace_kernel_stats(void* workspace, int reset, fp4
   return FP4_OK;
 }
 
-extern "C" fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out, void* stream) {
+extern "C" fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, int64_t pair, uint8_t* out,
+                                     void* stream) {
   int64_t n;
   FP4_TRY(checked_count({rows, k}, &n));
-  if (rows % 128 != 0 || k % 128 != 0) return FP4_ERR_UNSUPPORTED;
+  if (pair < 0) return FP4_ERR_INVALID_ARG;
+  if (k % 128 != 0) return FP4_ERR_UNSUPPORTED;
+  if (pair == 0 && rows % 128 != 0) return FP4_ERR_UNSUPPORTED;
+  if (pair > 0 && (pair % 64 != 0 || rows % (2 * pair) != 0)) return FP4_ERR_UNSUPPORTED;
   if (scales == nullptr || out == nullptr) return FP4_ERR_INVALID_ARG;
   if (!aligned16(scales) || !aligned16(out)) return FP4_ERR_ALIGNMENT;
-  return launch_mma_scales(scales, rows, k, out, static_cast<cudaStream_t>(stream));
+  return launch_mma_scales(scales, rows, k, pair, out, static_cast<cudaStream_t>(stream));
 }

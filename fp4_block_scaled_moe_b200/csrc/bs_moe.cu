@@ -9,23 +9,25 @@
 // 2^-8 |x| per element.  The two terms of token slot i are B rows 2i and 2i + 1, so the
 // product with x_i is D[:, 2i] + D[:, 2i + 1].
 //
-// A work unit is (expert, tile, token group): two 128-row weight tiles A0 and A1 times
-// the group's activation rows, into two fp32 accumulators D0 and D1 in TMEM.  gate_up:
-// A0 = gate rows t*128.., A1 = the up rows of the same intermediate indices, so g and u
-// of one index sit in the same TMEM lane.  down: A0, A1 = output rows t*256.. and
-// t*256+128...
+// A work unit is (expert, tile, token group): one 128-row weight tile times the group's
+// activation rows (up to 224 = 112 slots x 2 terms) into one fp32 accumulator in TMEM.
+// Each M = 128, K = 32 MMA reads its 4 KB A tile from shared memory in about the time
+// of a 128 x 256 product, so the units carry as many columns as TMEM allows.  gate_up
+// tiles are 64 gate rows followed by the 64 up rows of the same intermediate indices;
+// down tiles are 128 output rows.
 //
 // Warp roles of one persistent CTA per SM:
-//   warp 0     producer: TMA of the two weight tiles (FP4 widened to 16-byte slots,
-//              128-byte swizzle) and of the activation-term tile, and one bulk copy per
-//              scale atom (weights: re-laid once by fp4_mma_scales or per call into the
-//              workspace; activations: written as atoms by their producers).
-//   warp 1     MMA issuer and TMEM owner: per stage, scales -> TMEM, then 2 x 4 MMAs of
-//              K = 32 into one of two double-buffered accumulator pairs.
-//   warps 2-5  epilogue, one TMEM lane quadrant each: term pairs summed; gate_up applies
-//              the SwiGLU clamp and writes h split again into two MXFP8 terms for the
-//              down GEMM; down scales rows by the gate weight and writes fp32 in slot
-//              order for the combine.
+//   warp 0     producer: TMA of the weight tile (two 64-row boxes, FP4 widened to
+//              16-byte slots, 128-byte swizzle) and of the activation-term tile, and one
+//              bulk copy per scale atom (weights: re-laid once by fp4_mma_scales or per
+//              call into the workspace; activations: written as atoms by their producers).
+//   warp 1     MMA issuer and TMEM owner: per stage, scales -> TMEM, then 4 MMAs of K = 32
+//              into one of two accumulators (double-buffered against the epilogue).
+//   warps 2-5  epilogue, one TMEM lane quadrant each: term pairs summed.  gate_up: the up
+//              warps hand their rows to the gate warps through shared memory; the gate
+//              warps apply the SwiGLU clamp and write h split again into two MXFP8 terms
+//              for the down GEMM.  down: rows scaled by the gate weight, written as fp32 in
+//              slot order for the combine.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -37,19 +39,19 @@ namespace {
 constexpr int kBsThreads = 6 * 32;
 constexpr int kBsMaxStages = 8;
 constexpr int kKT = 128;                  // K elements per stage (one 128-byte swizzle row of E4M3)
-constexpr int kATile = 128 * 128;         // shared bytes of one 128-row FP4 tile (16-byte slots)
-constexpr int kSfBytes = 3 * 512;         // scale atoms per stage: A0, A1, B
-constexpr int kSfCols = 16;               // TMEM columns per stage for scales (4 each)
-constexpr int kMaxTokCap = 56;            // tokens per unit: accumulators of 2 x 56 columns
+constexpr int kATile = 128 * 128;         // shared bytes of the 128-row FP4 tile (16-byte slots)
+constexpr int kSfBytes = 3 * 512;         // scale atoms per stage: A, B rows 0-127, B rows 128-255
+constexpr int kSfCols = 16;               // TMEM columns per stage for scales (A 4, B 8)
+constexpr int kMaxTokCap = 112;           // tokens per unit: accumulators of 224 columns
 constexpr int kMaxExperts = 1024;
 
 struct BsLayout {
   int ntok_cap;      // tokens per work unit
-  int ncols;         // columns per accumulator = rows of the B box (16-multiple, <= 112)
+  int ncols;         // columns per accumulator = rows of the B box (16-multiple, <= 224)
   int stage_bytes;
   int stages;
   int tmem_cols;
-  int cnt_off, off_off, pre_off, bar_off;
+  int xch_off, cnt_off, off_off, pre_off, bar_off;
   int smem_bytes;
 };
 
@@ -83,6 +85,10 @@ __device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* o
 __device__ __forceinline__ uint32_t sf_row_off(int r) {
   return static_cast<uint32_t>((r & 31) * 16 + (r >> 5) * 4);
 }
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// activation-term rows 0..255 of a token group span two atoms
+__device__ __forceinline__ uint32_t sf_row_off2(int r) { return static_cast<uint32_t>((r >> 7) * 512) + sf_row_off(r & 127); }
 
 // E4M3 byte (satfinite, round to nearest even) of y, and its exact value
 __device__ __forceinline__ uint32_t e4m3_rn(float y, float& back) {
@@ -215,23 +221,37 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
     d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
     d2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
     d2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
-    uint8_t* at = atoms + (gid * kb128 + (b >> 2)) * 512 + (b & 3);
-    at[sf_row_off(2 * i)] = static_cast<uint8_t>(e1 + 127);
-    at[sf_row_off(2 * i + 1)] = static_cast<uint8_t>(e2 + 127);
+    uint8_t* at = atoms + (gid * kb128 + (b >> 2)) * 1024 + (b & 3);
+    at[sf_row_off2(2 * i)] = static_cast<uint8_t>(e1 + 127);
+    at[sf_row_off2(2 * i + 1)] = static_cast<uint8_t>(e2 + 127);
   }
   pdl_launch_dependents();
 }
 
 // Weight scales [rows][K/32] -> atoms: one thread moves the 4-byte word of one row and
-// one 128-K block.
+// one 128-K block.  pair == 0: tiles are 128 consecutive rows.  pair == I: rows are the
+// gate_up rows of experts (2I rows each) and tile t of expert e is gate rows t*64 .. +63
+// followed by up rows I + t*64 .. +63.
 __global__ void __launch_bounds__(256) mma_scales_kernel(const uint8_t* __restrict__ scales, int64_t rows,
-                                                         int64_t K, uint8_t* __restrict__ atoms) {
+                                                         int64_t K, int64_t pair, uint8_t* __restrict__ atoms) {
   const int64_t kb = K / 128, total = rows * kb;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = idx / kb, c = idx % kb;
+    int64_t tile;
+    int within;
+    if (pair == 0) {
+      tile = r >> 7;
+      within = static_cast<int>(r & 127);
+    } else {
+      const int64_t e = r / (2 * pair), rl = r % (2 * pair);
+      const bool up = rl >= pair;
+      const int64_t q = up ? rl - pair : rl;
+      tile = e * (pair / 64) + q / 64;
+      within = static_cast<int>(q % 64) + (up ? 64 : 0);
+    }
     const uint32_t w = *reinterpret_cast<const uint32_t*>(scales + r * (K / 32) + 4 * c);
-    *reinterpret_cast<uint32_t*>(atoms + ((r >> 7) * kb + c) * 512 + sf_row_off(static_cast<int>(r & 127))) = w;
+    *reinterpret_cast<uint32_t*>(atoms + (tile * kb + c) * 512 + sf_row_off(within)) = w;
   }
 }
 
@@ -257,7 +277,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   int* off = reinterpret_cast<int*>(smem + L.off_off);
   int* pre = reinterpret_cast<int*>(smem + L.pre_off);
   const int E = a.E;
-  const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 128 : a.rows_per_expert / 256;
+  const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 64 : a.rows_per_expert / 128;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -317,7 +337,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   const int n_units = pre[E];
   const int nk = a.K / kKT;
   const uint32_t stg = static_cast<uint32_t>(L.stage_bytes);
-  const uint32_t b_off = 2 * kATile, sf_off = 2 * kATile + L.ncols * kKT;   // within a stage
+  const uint32_t b_off = kATile, sf_off = kATile + L.ncols * kKT;   // within a stage
 
   if (warp == 0) {
     // ------------------------------------ producer ------------------------------------
@@ -337,12 +357,13 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       }
       const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
       const int64_t rbase = static_cast<int64_t>(un.e) * a.rows_per_expert;
-      const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 128 : rbase + un.tile * 256;
-      const int64_t y1 = (kEpi == kEpiSwiglu) ? y0 + a.inter : y0 + 128;
+      const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 64 : rbase + un.tile * 128;
+      const int64_t y1 = (kEpi == kEpiSwiglu) ? y0 + a.inter : y0 + 64;
       const int brow0 = 2 * un.slot0;
-      const uint8_t* sa0 = a.a_atoms + (y0 >> 7) * nk * 512;
-      const uint8_t* sa1 = a.a_atoms + (y1 >> 7) * nk * 512;
-      const uint8_t* sb = a.b_atoms + static_cast<int64_t>(un.gid) * nk * 512;
+      const int64_t tile_g = static_cast<int64_t>(un.e) * tiles + un.tile;      // tile across experts
+      const uint8_t* sa = a.a_atoms + tile_g * nk * 512;
+      const uint8_t* sb = a.b_atoms + static_cast<int64_t>(un.gid) * nk * 1024;
+      const bool two_b = 2 * un.ntok > 128;
       for (int c = 0; c < nk; ++c, ++it) {
         const int s = it % S;
         if (it >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / S) & 1) ^ 1, a.status))) {
@@ -353,12 +374,12 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         const uint32_t st = sbase + s * stg;
         const uint32_t sf = st + sf_off;
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(2 * 128 * kKT / 2 + L.ncols * kKT + kSfBytes));
-          bulk_g2s(sf, sa0 + c * 512, 512, bar_full + 8 * s);
-          bulk_g2s(sf + 512, sa1 + c * 512, 512, bar_full + 8 * s);
-          bulk_g2s(sf + 1024, sb + c * 512, 512, bar_full + 8 * s);
+          const uint32_t sfb = two_b ? 1024u : 512u;
+          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(128 * kKT / 2 + L.ncols * kKT) + 512u + sfb);
+          bulk_g2s(sf, sa + c * 512, 512, bar_full + 8 * s);
+          bulk_g2s(sf + 512, sb + c * 1024, sfb, bar_full + 8 * s);
           tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * s);
-          tma_load_2d(st + kATile, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
+          tma_load_2d(st + kATile / 2, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
           tma_load_2d(st + b_off, &tmB, c * kKT, brow0, bar_full + 8 * s);
         }
         __syncwarp();
@@ -375,7 +396,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------ MMA issuer ----------------------------------
-    const uint32_t sf_t0 = tmem + static_cast<uint32_t>(4 * L.ncols);
+    const uint32_t sf_t0 = tmem + static_cast<uint32_t>(2 * L.ncols);
     int it = 0, uc = 0;
     bool ok = true;
     while (ok) {
@@ -395,7 +416,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
       const uint32_t N = static_cast<uint32_t>((2 * un.ntok + 15) & ~15);
       const uint32_t idesc = tc::idesc_mxf8f6f4(5u, 0u, 128u, N);
-      const uint32_t d0 = tmem + static_cast<uint32_t>(buf * 2 * L.ncols), d1 = d0 + static_cast<uint32_t>(L.ncols);
+      const uint32_t d0 = tmem + static_cast<uint32_t>(buf * L.ncols);
       for (int c = 0; c < nk; ++c, ++it) {
         const int s = it % S;
         if (c > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s, (it / S) & 1, a.status))) {
@@ -409,15 +430,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           const uint32_t t0 = sf_t0 + s * kSfCols;
           tc::cp_sf_32x128b_x4(t0, tc::desc_k_interleave(sf));
           tc::cp_sf_32x128b_x4(t0 + 4, tc::desc_k_interleave(sf + 512));
-          tc::cp_sf_32x128b_x4(t0 + 8, tc::desc_k_interleave(sf + 1024));
+          if (N > 128) tc::cp_sf_32x128b_x4(t0 + 8, tc::desc_k_interleave(sf + 1024));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t bd = tc::desc_k_sw128(st + b_off + 32 * j);
-            const uint32_t acc = static_cast<uint32_t>((c | j) != 0);
-            tc::mma_mxf8f6f4(d0, tc::desc_k_sw128(st + 32 * j), bd, idesc, t0, t0 + 8, static_cast<uint32_t>(j), acc);
-            tc::mma_mxf8f6f4(d1, tc::desc_k_sw128(st + kATile + 32 * j), bd, idesc, t0 + 4, t0 + 8,
-                             static_cast<uint32_t>(j), acc);
-          }
+          for (int j = 0; j < 4; ++j)
+            tc::mma_mxf8f6f4(d0, tc::desc_k_sw128(st + 32 * j), tc::desc_k_sw128(st + b_off + 32 * j), idesc, t0,
+                             t0 + 4, static_cast<uint32_t>(j), static_cast<uint32_t>((c | j) != 0));
           tc::commit(bar_empty + 8 * s);
           if (c == nk - 1) tc::commit(bar_accf + 8 * buf);
         }
@@ -432,7 +449,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   } else {
     // ------------------------------------ epilogue -------------------------------------
     const int q = warp & 3;                    // TMEM lane quadrant this warp may access
-    const int row = 32 * q + lane;             // accumulator row within each 128-row tile
+    const int row = 32 * q + lane;             // accumulator row = row of the weight tile
+    float* xch = reinterpret_cast<float*>(smem + L.xch_off);   // [2][64][8]: up values for the gate warps
     int uc = 0;
     while (true) {
       const int buf = uc & 1;
@@ -442,60 +460,69 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       tc::fence_after_sync();
       const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
       const uint32_t d0 =
-          tmem + static_cast<uint32_t>(buf * 2 * L.ncols) + (static_cast<uint32_t>(32 * q) << 16);
-      const uint32_t d1 = d0 + static_cast<uint32_t>(L.ncols);
+          tmem + static_cast<uint32_t>(buf * L.ncols) + (static_cast<uint32_t>(32 * q) << 16);
       const int N = (2 * un.ntok + 15) & ~15;
       if (kEpi == kEpiSwiglu) {
-        const int64_t col = static_cast<int64_t>(un.tile) * 128 + row;
-        uint8_t* hat = a.h_atoms + (static_cast<int64_t>(un.gid) * (a.inter / 128) + un.tile) * 512 + q;
+        // rows 0-63 gate, 64-127 up of intermediate indices tile*64 + (row & 63)
+        const int64_t col = static_cast<int64_t>(un.tile) * 64 + (row & 63);
+        uint8_t* hat = a.h_atoms + (static_cast<int64_t>(un.gid) * (a.inter / 128) + (col >> 7)) * 1024 +
+                       ((col & 127) >> 5);
         for (int c0 = 0; c0 < N; c0 += 16) {
-          uint32_t vg[16], vu[16];
-          tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), vg);
-          tc::ld_32x32b_x16(d1 + static_cast<uint32_t>(c0), vu);
+          float* xb = xch + ((c0 >> 4) & 1) * (64 * 8);
+          uint32_t v[16];
+          tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), v);
           tc::ld_wait();
+          if (q >= 2) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int i = (c0 >> 1) + j;
-            const float g = fminf(__uint_as_float(vg[2 * j]) + __uint_as_float(vg[2 * j + 1]), a.limit);
-            const float uu = fminf(fmaxf(__uint_as_float(vu[2 * j]) + __uint_as_float(vu[2 * j + 1]), -a.limit), a.limit);
-            const float hv = __fdividef(g, 1.0f + __expf(-g)) * uu;
-            uint32_t q1, q2, s1, s2;
-            warp_split2(hv, q1, q2, s1, s2);
-            if (i < un.ntok) {
-              const int64_t r0 = 2 * (static_cast<int64_t>(un.slot0) + i);
-              a.hq[r0 * a.inter + col] = static_cast<uint8_t>(q1);
-              a.hq[(r0 + 1) * a.inter + col] = static_cast<uint8_t>(q2);
-              if (lane == 0) {
-                hat[sf_row_off(2 * i)] = static_cast<uint8_t>(s1);
-                hat[sf_row_off(2 * i + 1)] = static_cast<uint8_t>(s2);
+            for (int j = 0; j < 8; ++j)
+              xb[(row - 64) * 8 + j] = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+          }
+          epi_bar_sync();
+          if (q < 2) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int i = (c0 >> 1) + j;
+              const float g = fminf(__uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]), a.limit);
+              const float uu = fminf(fmaxf(xb[row * 8 + j], -a.limit), a.limit);
+              const float hv = __fdividef(g, 1.0f + __expf(-g)) * uu;
+              uint32_t q1, q2, s1, s2;
+              warp_split2(hv, q1, q2, s1, s2);
+              if (i < un.ntok) {
+                const int64_t r0 = 2 * (static_cast<int64_t>(un.slot0) + i);
+                a.hq[r0 * a.inter + col] = static_cast<uint8_t>(q1);
+                a.hq[(r0 + 1) * a.inter + col] = static_cast<uint8_t>(q2);
+                if (lane == 0) {
+                  hat[sf_row_off2(2 * i)] = static_cast<uint8_t>(s1);
+                  hat[sf_row_off2(2 * i + 1)] = static_cast<uint8_t>(s2);
+                }
               }
             }
           }
         }
       } else {
-        // gate weights of the unit's tokens, one per lane (ntok <= 64)
-        const float w_lo = (lane < un.ntok) ? a.gw[a.perm[un.slot0 + lane]] : 0.f;
-        const float w_hi = (lane + 32 < un.ntok) ? a.gw[a.perm[un.slot0 + 32 + lane]] : 0.f;
-        float* o0 = a.o_out + static_cast<int64_t>(un.slot0) * a.ldo + static_cast<int64_t>(un.tile) * 256 + row;
+        // gate weights of the unit's tokens (ntok <= 128): lane l holds slots l, 32+l, 64+l, 96+l
+        float wl[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int i = lane + 32 * m;
+          wl[m] = (i < un.ntok) ? a.gw[a.perm[un.slot0 + i]] : 0.f;
+        }
+        float* o0 = a.o_out + static_cast<int64_t>(un.slot0) * a.ldo + static_cast<int64_t>(un.tile) * 128 + row;
         for (int c0 = 0; c0 < N; c0 += 16) {
-          uint32_t v0[16], v1[16];
-          tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), v0);
-          tc::ld_32x32b_x16(d1 + static_cast<uint32_t>(c0), v1);
+          uint32_t v[16];
+          tc::ld_32x32b_x16(d0 + static_cast<uint32_t>(c0), v);
           tc::ld_wait();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int i = (c0 >> 1) + j;
-            const float wgt = __shfl_sync(0xFFFFFFFFu, (i < 32) ? w_lo : w_hi, i & 31);
-            if (i < un.ntok) {
-              float* o = o0 + static_cast<int64_t>(i) * a.ldo;
-              o[0] = (__uint_as_float(v0[2 * j]) + __uint_as_float(v0[2 * j + 1])) * wgt;
-              o[128] = (__uint_as_float(v1[2 * j]) + __uint_as_float(v1[2 * j + 1])) * wgt;
-            }
+            const float wsel = (i < 32) ? wl[0] : (i < 64) ? wl[1] : (i < 96) ? wl[2] : wl[3];
+            const float wgt = __shfl_sync(0xFFFFFFFFu, wsel, i & 31);
+            if (i < un.ntok) o0[static_cast<int64_t>(i) * a.ldo] = (__uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1])) * wgt;
           }
         }
       }
       tc::fence_before_sync();
-      __syncwarp();
+      epi_bar_sync();
       if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
       ++uc;
     }
@@ -514,9 +541,11 @@ constexpr int kBsSmemLimit = 227 * 1024;
 bool bs_layout(int T, int E, BsLayout* L) {
   L->ntok_cap = std::min(kMaxTokCap, (T + 7) / 8 * 8);
   L->ncols = (2 * L->ntok_cap + 15) / 16 * 16;
-  L->stage_bytes = static_cast<int>(align_up(static_cast<size_t>(2 * kATile + L->ncols * kKT + kSfBytes), 1024));
-  // fixed part (after the stages): per-expert tables, barriers
+  L->stage_bytes = static_cast<int>(align_up(static_cast<size_t>(kATile + L->ncols * kKT + kSfBytes), 1024));
+  // fixed part (after the stages): exchange buffer, per-expert tables, barriers
   int off = 0;
+  const int x0 = off;
+  off += 2 * 64 * 8 * 4;
   const int c0 = off;
   off += 4 * (E + 1);
   const int o0 = off;
@@ -529,16 +558,17 @@ bool bs_layout(int T, int E, BsLayout* L) {
   const int fixed = static_cast<int>(align_up(off, 16));
   int S = (kBsSmemLimit - 1024 - fixed) / L->stage_bytes;
   S = std::min(S, kBsMaxStages);
-  while (S > 0 && 4 * L->ncols + kSfCols * S > 512) --S;
+  while (S > 0 && 2 * L->ncols + kSfCols * S > 512) --S;
   if (S < 2) return false;
   L->stages = S;
   const int body = S * L->stage_bytes;
+  L->xch_off = body + x0;
   L->cnt_off = body + c0;
   L->off_off = body + o0;
   L->pre_off = body + p0;
   L->bar_off = body + b0;
   L->smem_bytes = body + fixed + 1024;      // + slack for the 1024-byte alignment of the base
-  const int need = 4 * L->ncols + kSfCols * S;
+  const int need = 2 * L->ncols + kSfCols * S;
   int cols = 32;
   while (cols < need) cols *= 2;
   L->tmem_cols = cols;
@@ -555,10 +585,11 @@ fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t*
                     ntok_cap, q, atoms);
 }
 
-fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st) {
+fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, int64_t pair, uint8_t* atoms,
+                             cudaStream_t st) {
   const int64_t total = rows * (K / 128);
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, num_sms() * 16)));
-  mma_scales_kernel<<<grid, 256, 0, st>>>(scales, rows, K, atoms);
+  mma_scales_kernel<<<grid, 256, 0, st>>>(scales, rows, K, pair, atoms);
   FP4_TRY_CUDA(cudaGetLastError());
   note_launch();
   return FP4_OK;
@@ -571,12 +602,12 @@ int bs_ntok_cap(int T, int E) {
 
 size_t bs_group_atom_bytes(int P, int E, int ntok_cap, int K) {
   const size_t groups = static_cast<size_t>(P) / ntok_cap + E + 1;   // >= sum over experts of ceil(n_e / cap)
-  return groups * (K / 128) * 512;
+  return groups * (K / 128) * 1024;
 }
 
 bool bs_supported(int T, int E, int H, int I) {
   BsLayout L;
-  return H % 256 == 0 && I % 128 == 0 && bs_layout(T, E, &L);
+  return H % 128 == 0 && I % 128 == 0 && bs_layout(T, E, &L);
 }
 
 fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
@@ -584,7 +615,7 @@ fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
   if (!bs_layout(T, a.E, &L) || L.ntok_cap != a.ntok_cap) return FP4_ERR_UNSUPPORTED;
   CUtensorMap mA, mB;
   FP4_TRY(make_tmap_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.codes, static_cast<uint64_t>(a.K),
-                       static_cast<uint64_t>(a.rows_total), static_cast<uint64_t>(a.K / 2), kKT, 128,
+                       static_cast<uint64_t>(a.rows_total), static_cast<uint64_t>(a.K / 2), kKT, 64,
                        CU_TENSOR_MAP_SWIZZLE_128B));
   FP4_TRY(make_tmap_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_q, static_cast<uint64_t>(a.K),
                        static_cast<uint64_t>(2) * a.P, static_cast<uint64_t>(a.K), kKT,

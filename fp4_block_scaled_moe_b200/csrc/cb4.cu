@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(1024) cb4_scan_kernel(int32_t* __restrict__ ro
   __shared__ int32_t part[1024];
   const int tid = threadIdx.x;
   const int64_t per = (rows + 1023) / 1024;
-  const int64_t r0 = 1 + tid * per, r1 = std::min<int64_t>(rows + 1, r0 + per);
+  const int64_t r0 = 1 + tid * per, r1 = (r0 + per < rows + 1) ? r0 + per : rows + 1;
   int32_t s = 0;
   for (int64_t r = r0; r < r1; ++r) s += row_ptr[r];
   part[tid] = s;

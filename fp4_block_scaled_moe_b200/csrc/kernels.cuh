@@ -108,11 +108,12 @@ __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __res
 // Block-scaled tensor-core expert GEMM (MXFP4 weights x two-term MXFP8 activations).
 // Scale atoms: 512 bytes holding the UE8M0 scales of 128 rows x 128 K (four 32-blocks):
 // row r, block b at byte (r % 32) * 16 + (r / 32) * 4 + b -- the layout the TMEM scale
-// copy (tcgen05.cp 32x128b, warpx4) reads.  Weights: atom (row block, K block) at
-// ((row / 128) * (K / 128) + k / 128) * 512.  Activation terms: one atom per (token
-// group, K block) at (group * (K / 128) + k / 128) * 512, rows 2i, 2i + 1 = the two
-// terms of the group's i-th slot; groups are the per-expert runs of ntok_cap slots,
-// numbered across experts in expert order.
+// copy (tcgen05.cp 32x128b, warpx4) reads.  Weights: atom (tile, K block) at
+// (tile * (K / 128) + k / 128) * 512, a tile being 128 consecutive rows (down) or the
+// 64 gate rows and 64 matching up rows of one expert (gate_up).  Activation terms: two
+// atoms (rows 0-127, 128-255) per (token group, K block) at (group * (K / 128) + k / 128)
+// * 1024, rows 2i, 2i + 1 = the two terms of the group's i-th slot; groups are the
+// per-expert runs of ntok_cap slots, numbered across experts in expert order.
 struct BsArgs {
   int epi;                        // kEpiSwiglu (gate_up + SwiGLU) or kEpiDown
   const uint8_t* codes;           // A: [rows_total][K/2] E2M1 pairs
@@ -142,7 +143,9 @@ struct BsArgs {
 int bs_ntok_cap(int T, int E);
 // bytes of the activation scale atoms for P slots over E experts at this K
 size_t bs_group_atom_bytes(int P, int E, int ntok_cap, int K);
-fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st);
+// pair = 0: tiles of 128 consecutive rows; pair = I: gate_up tiles of 64 gate + 64 up rows
+fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, int64_t pair, uint8_t* atoms,
+                             cudaStream_t st);
 bool bs_supported(int T, int E, int H, int I);
 fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st);
 fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t* counts, const int32_t* offsets,

@@ -157,11 +157,11 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     const uint8_t* agu = w->gu_mma_scales;
     const uint8_t* adn = w->dn_mma_scales;
     if (agu == nullptr) {
-      FP4_TRY(launch_mma_scales(w->gu_scales, static_cast<int64_t>(E) * 2 * I, H, ws + L.agu, st));
+      FP4_TRY(launch_mma_scales(w->gu_scales, static_cast<int64_t>(E) * 2 * I, H, I, ws + L.agu, st));
       agu = ws + L.agu;
     }
     if (adn == nullptr) {
-      FP4_TRY(launch_mma_scales(w->dn_scales, static_cast<int64_t>(E) * H, I, ws + L.adn, st));
+      FP4_TRY(launch_mma_scales(w->dn_scales, static_cast<int64_t>(E) * H, I, 0, ws + L.adn, st));
       adn = ws + L.adn;
     }
     FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, ra.counts, ra.offsets, E, k, P, H, cap, xq,

@@ -197,14 +197,17 @@ typedef struct fp4_moe_weights {
 
 /*
  * fp4_mma_scales: MXFP4 scales [rows, k/32] (UE8M0, row-major, as fp4_pack writes them)
- * re-laid for the tensor-core expert kernels: one 512-byte atom per 128 rows x 128 k,
- * atom (row/128, k/128) at ((row/128) * (k/128) + k/128) * 512, scale of row r and
- * 32-block b inside it at (r % 32) * 16 + ((r % 128) / 32) * 4 + b % 4 -- the order the
- * tensor-memory scale copy reads.  out: rows * k / 32 bytes.  rows % 128 == 0 and
- * k % 128 == 0 (else FP4_ERR_UNSUPPORTED); pointers 16-byte aligned.  No counterpart
- * in the pages: a layout of this library's MMA kernels.
+ * re-laid for the tensor-core expert kernels: one 512-byte atom per tile of 128 rows and
+ * 128 k, atom (tile, k/128) at (tile * (k/128) + k/128) * 512, the scale of tile row r
+ * and 32-block b inside it at (r % 32) * 16 + (r / 32) * 4 + b % 4 -- the order the
+ * tensor-memory scale copy reads.  pair = 0: tile t = rows 128t .. 128t+127 (down
+ * weights; rows % 128 == 0).  pair = I > 0: rows are gate_up rows of experts with 2I rows
+ * each (rows % 2I == 0, I % 64 == 0) and tile (e, t) = gate rows t*64 .. t*64+63 followed
+ * by up rows I + t*64 .. I + t*64+63 of expert e, numbered e * (I/64) + t.  k % 128 == 0.
+ * out: rows * k / 32 bytes.  FP4_ERR_UNSUPPORTED on other shapes; pointers 16-byte
+ * aligned.  No counterpart in the pages: a layout of this library's MMA kernels.
  */
-fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out, void* stream);
+fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, int64_t pair, uint8_t* out, void* stream);
 
 /* Optional copies of the routing results of a forward call (each pointer may be NULL). */
 typedef struct fp4_route_out {
