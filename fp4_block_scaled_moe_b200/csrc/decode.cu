@@ -1,7 +1,7 @@
 // Grouped W4A16 GEMV for the decode path: few tokens per expert, so the layer is
 // bound by the weight stream from HBM.
 //
-// Design (B200): persistent CTAs, two per SM, walk work units {expert, 64-row weight
+// Design (B200): persistent CTAs, two or three per SM, walk work units {expert, 64-row weight
 // tile, up to 8 routed tokens}.  One producer warp streams a unit's 4-bit codes with TMA
 // (128-byte swizzled boxes, conflict-free for the fragment reads), its scale bytes with
 // 4-byte async copies and the f16 activation rows with 1D bulk copies into a shared-
@@ -40,7 +40,10 @@ constexpr int kConsumers = 8;             // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kRedPitch = kTok + 1;       // fp32 reduction row pitch
-constexpr int kSmemBudget = 110 * 1024;   // two CTAs per SM
+// CTAs per SM: stages 512 K wide run two per SM (110 KB of shared memory each), 256 K
+// wide ones three (73 KB each, at most 72 registers a thread)
+constexpr int ctas_per_sm(int kc) { return kc == 256 ? 3 : 2; }
+constexpr int smem_budget(int kc) { return kc == 256 ? 73 * 1024 : 110 * 1024; }
 
 struct Layout {
   int kc;            // K elements per stage
@@ -55,6 +58,8 @@ struct Layout {
   int lut_off;       // 256 fp32 (UE8M0 -> float)
   int cnt_off, off_off, pre_off;   // [E + 1] int each (pre is followed by [E] cursors)
   int perm_off;      // [P] int (kModeRoute)
+  int scl_off;       // [scl_n] float: per-slot epilogue factor (2^sexp or gate weight)
+  int scl_n;         // slots with a preloaded factor (0: read per unit from global memory)
   int bar_off;
   int smem_bytes;
 };
@@ -170,7 +175,7 @@ __device__ __forceinline__ void cb4_lookup8(uint32_t w, const uint32_t (&lo)[4],
 }
 
 template <int kFmt, int kEpi, int kMode, int KC>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a, const Layout L) {
   // stage geometry (must match make_layout)
   constexpr int kB = (kFmt == FP4_MXFP4) ? 32 : 16;
@@ -379,6 +384,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t s_off = kScalesOff + rbase * kScaleRow +
                          (kFmt == FP4_MXFP4 ? jbase : (kFmt == FP4_NVFP4 ? 2 * jbase : (jbase >> 2) * 32));
   const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
+  // per-slot epilogue factors, loaded once so no unit's epilogue waits on global memory
+  float* scl_s = reinterpret_cast<float*>(smem + L.scl_off);
+  if (L.scl_n > 0) {
+    for (int i = threadIdx.x; i < L.scl_n; i += kConsumers * 32) {
+      float v;
+      if (kEpi == kEpiSwiglu) v = ldexpf(1.0f, a.sexp[perm_at(i) / a.topk]);
+      else if (kEpi == kEpiDown) v = a.gw[perm_at(i)];
+      else v = ldexpf(1.0f, a.sexp[i]);
+      scl_s[i] = v;
+    }
+    named_bar_sync();
+  }
   int it = 0;
   while (true) {
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * (it % L.stages), (it / L.stages) & 1, a.status))) {
@@ -388,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int u = *reinterpret_cast<volatile int*>(&stage_unit[it % L.stages]);
     if (u < 0) break;                              // sentinel: no more work
     const Unit un = get_unit(u);
+    const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e] : 1.0f;   // used after the K loop
     float acc[2][4];
 #pragma unroll
     for (int m = 0; m < 2; ++m)
@@ -511,7 +529,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       return ((red[o] + red[q + o]) + red[2 * q + o]) + red[3 * q + o];
     };
     // ---- fused epilogue ----
-    const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e] : 1.0f;
     // CB4 sparse term of row r against an activation row (same scaling as the MMA input)
     auto sparse = [&](int r, const __half* xrow) -> float {
       if (kFmt != FP4_CB4 || a.sp_rowptr == nullptr) return 0.f;
@@ -524,9 +541,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (kEpi == kEpiSwiglu) {
       for (int idx = threadIdx.x; idx < 32 * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 31, i = idx >> 5;
-        const int tok = perm_at(un.slot0 + i) / a.topk;
-        const float sc = ldexpf(ts, a.sexp[tok]);
-        const __half* xrow = a.x16 + static_cast<int64_t>(tok) * a.K;
+        const float sc = (L.scl_n > 0) ? ts * scl_s[un.slot0 + i]
+                                       : ldexpf(ts, a.sexp[perm_at(un.slot0 + i) / a.topk]);
+        const __half* xrow =
+            (kFmt == FP4_CB4) ? a.x16 + static_cast<int64_t>(perm_at(un.slot0 + i) / a.topk) * a.K : nullptr;
         const float gv = fminf((val(r, i) + sparse(r, xrow)) * sc, a.limit);
         const float uv = fminf(fmaxf((val(32 + r, i) + sparse(32 + r, xrow)) * sc, -a.limit), a.limit);
         const float hv = gv / (1.0f + expf(-gv)) * uv;
@@ -535,14 +553,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else if (kEpi == kEpiDown) {
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
-        const float wgt = a.gw[perm_at(un.slot0 + i)];
+        const float wgt = (L.scl_n > 0) ? scl_s[un.slot0 + i] : a.gw[perm_at(un.slot0 + i)];
         const float v = val(r, i) + sparse(r, a.x16 + static_cast<int64_t>(un.slot0 + i) * a.K);
         a.o_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] = v * ts * wgt;
       }
     } else {
       for (int idx = threadIdx.x; idx < kRows * un.ntok; idx += kConsumers * 32) {
         const int r = idx & 63, i = idx >> 6;
-        const float v = ldexpf(val(r, i) * ts, a.sexp[un.slot0 + i]);
+        const float v = (L.scl_n > 0) ? (val(r, i) * ts) * scl_s[un.slot0 + i]
+                                      : ldexpf(val(r, i) * ts, a.sexp[un.slot0 + i]);
         a.y_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] =
             __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
@@ -551,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   finish();
 }
 
-Layout make_layout(int fmt, int K, int E, int P) {
+Layout make_layout(int fmt, int K, int E, int P, int P_scl) {
   Layout L{};
   const int B = (fmt == FP4_MXFP4) ? 32 : 16;
   // CB4 stages carry 4 codebook bytes per 16 indices: the smaller stage keeps 5 in flight
@@ -568,8 +587,10 @@ Layout make_layout(int fmt, int K, int E, int P) {
   const int Eb = static_cast<int>(align_up(sizeof(int) * (E + 1), 16));
   const int Cb = static_cast<int>(align_up(sizeof(int) * E, 16));
   const int Pb = static_cast<int>(align_up(sizeof(int) * P, 16));
-  const int fixed = 4 * kRows * kRedPitch * 4 + 4 * kMaxStages + 1024 + 3 * Eb + Cb + Pb + 16 * kMaxStages + 1024;
-  L.stages = std::min(kMaxStages, (kSmemBudget - fixed) / L.stage_bytes);
+  const int Sb = static_cast<int>(align_up(sizeof(float) * P_scl, 16));
+  const int fixed =
+      4 * kRows * kRedPitch * 4 + 4 * kMaxStages + 1024 + 3 * Eb + Cb + Pb + Sb + 16 * kMaxStages + 1024;
+  L.stages = std::min(kMaxStages, (smem_budget(kc) - fixed) / L.stage_bytes);
   if (L.stages < 2 || L.stages * L.stage_bytes < static_cast<int>(sizeof(int)) * P) return Layout{};
   L.red_off = L.stages * L.stage_bytes;
   L.su_off = L.red_off + 4 * kRows * kRedPitch * 4;
@@ -578,7 +599,9 @@ Layout make_layout(int fmt, int K, int E, int P) {
   L.off_off = L.cnt_off + Eb;
   L.pre_off = L.off_off + Eb;
   L.perm_off = L.pre_off + Eb + Cb;
-  L.bar_off = L.perm_off + Pb;
+  L.scl_off = L.perm_off + Pb;
+  L.scl_n = P_scl;
+  L.bar_off = L.scl_off + Sb;
   L.smem_bytes = L.bar_off + 16 * kMaxStages + 1024;   // + alignment slack
   return L;
 }
@@ -618,13 +641,14 @@ fp4_status dispatch(const DecodeArgs& a, const Layout& L, const CUtensorMap& map
 
 fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
   const int E = (a.mode == kModeStatic) ? 1 : a.E;
-  const int P = (a.mode == kModeRoute) ? a.T * a.topk : 0;
-  const Layout L = make_layout(a.fmt, a.K, E, P);
+  const int P_all = (a.mode == kModeStatic) ? a.T : a.T * a.topk;
+  const int P = (a.mode == kModeRoute) ? P_all : 0;
+  const Layout L = make_layout(a.fmt, a.K, E, P, P_all <= kRouteMaxPairs ? P_all : 0);
   if (L.kc == 0) return FP4_ERR_UNSUPPORTED;
   CUtensorMap map;
   FP4_TRY(make_tmap_2d_u8(&map, a.codes, static_cast<uint64_t>(a.K / 2), static_cast<uint64_t>(a.rows_total),
                           static_cast<uint64_t>(a.K / 2), 128, 32, CU_TENSOR_MAP_SWIZZLE_128B));
-  int grid = 2 * num_sms();
+  int grid = ctas_per_sm(L.kc) * num_sms();
   if (a.mode == kModeStatic) grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok));
   if (a.fmt == FP4_CB4) return dispatch<FP4_CB4>(a, L, map, grid, st, pdl);
   return (a.fmt == FP4_NVFP4) ? dispatch<FP4_NVFP4>(a, L, map, grid, st, pdl)
