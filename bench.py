@@ -343,8 +343,8 @@ def oracle_sample(cfg, n_tokens):
 # gate_up bs_moe_kernel captured at a quarter of the experts and tokens and scaled by the
 # four times as many work units of the full layer.  None when no capture matches.
 NCU_TRAFFIC = {
-    ("moe_mxfp4_decode_e64_h2048_i768_k8_t16", "decode_kernel<gate_up+swiglu>"): 101_306_368,
-    ("moe_mxfp4_prefill_e256_h6144_i2048_k8_t8192", "bs_moe_kernel<gate_up+swiglu>"): 4 * 1_137_554_392,
+    ("moe_mxfp4_decode_e64_h2048_i768_k8_t16", "decode_kernel<gate_up+swiglu>"): 100_664_576,
+    ("moe_mxfp4_prefill_e256_h6144_i2048_k8_t8192", "bs_moe_kernel<gate_up+swiglu>"): 4 * 1_134_384_488,
 }
 
 

@@ -54,6 +54,7 @@ SIGNATURES = {
     "fp4_last_error_string": (ctypes.c_char_p, []),
     "fp4_version": (ctypes.c_char_p, []),
     "fp4_launch_count": (ctypes.c_ulonglong, []),
+    "fp4_selftest_wait_timeout": (_cint, [_vp, _i64, _vp]),
     "fp4_pack": (_cint, [_cint, _vp, _cint, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "fp4_mma_scales": (_cint, [_vp, _i64, _i64, _i64, _vp, _vp]),
     "fp4_cb4_row_ptr": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp]),

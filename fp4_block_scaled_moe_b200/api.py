@@ -247,6 +247,12 @@ def fp4_launch_count() -> int:
     return int(L.load().fp4_launch_count())
 
 
+def fp4_selftest_wait_timeout(workspace, limit_ns: int = 1_000_000):
+    """Run the bounded-wait failure path once (see include/fp4moe.h)."""
+    L.check("fp4_selftest_wait_timeout", L.load().fp4_selftest_wait_timeout(_ptr(workspace), int(limit_ns),
+                                                                           _stream(workspace.device)))
+
+
 def fp4_workspace_status(workspace) -> str:
     code = L.load().fp4_workspace_status(_ptr(workspace), _stream(workspace.device))
     return L.STATUS.get(code, str(code))

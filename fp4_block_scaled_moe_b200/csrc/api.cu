@@ -152,3 +152,32 @@ extern "C" fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_
   if (!aligned16(scales) || !aligned16(out)) return FP4_ERR_ALIGNMENT;
   return launch_mma_scales(scales, rows, k, pair, out, static_cast<cudaStream_t>(stream));
 }
+
+namespace fp4 {
+namespace {
+// One CTA waits on an mbarrier phase that nothing completes; the bounded wait gives up
+// after limit_ns, records the timeout in the status word and the kernel returns.
+__global__ void wait_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_for(b, 0, status, limit_ns);
+}
+}  // namespace
+}  // namespace fp4
+
+extern "C" fp4_status fp4_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream) {
+  if (workspace == nullptr) return FP4_ERR_INVALID_ARG;
+  if (limit_ns <= 0 || limit_ns > 2000000000ll) return FP4_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP4_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  wait_selftest_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t*>(workspace),
+                                         static_cast<unsigned long long>(limit_ns));
+  FP4_TRY_CUDA(cudaGetLastError());
+  note_launch();
+  return FP4_OK;
+}

@@ -130,19 +130,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase. On expiry records kStatusTimeout in *status and
-// returns false; the caller then stops issuing work and leaves.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
+// Bounded wait on an mbarrier phase. After limit_ns of %globaltimer records
+// kStatusTimeout in *status and returns false; the caller then stops issuing work and
+// leaves.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint32_t* status,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       if (status) atomicOr(status, kStatusTimeout);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
+  return mbar_wait_for(bar, parity, status, kWaitLimitNs);
 }
 
 // 1D bulk copy global -> shared, completion counted on an mbarrier (bytes % 16 == 0).

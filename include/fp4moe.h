@@ -264,6 +264,17 @@ fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K, 
 fp4_status fp4_workspace_status(const void* workspace, void* stream);
 
 /*
+ * fp4_selftest_wait_timeout: exercises the failure path of the library's bounded device
+ * waits without faulting the GPU.  Launches one kernel that waits on a shared-memory
+ * barrier phase nothing completes; after limit_ns (1 .. 2e9) of device time the wait
+ * gives up, sets the timeout bit in the status word of `workspace` (a workspace of
+ * moe_fp4_forward, 256-byte aligned) and the kernel returns.  fp4_workspace_status then
+ * reports FP4_ERR_TIMEOUT and clears the word; the context stays usable.  No
+ * counterpart in the pages.
+ */
+fp4_status fp4_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
+
+/*
  * moe_fp4_forward_noalloc: the same layer as moe_fp4_forward, for callers that cannot
  * allocate device memory (no counterpart in the pages: an addition of this library).
  * Some callers have no way to provide a workspace: a CUDA graph captured once that must

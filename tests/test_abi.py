@@ -106,6 +106,13 @@ def test_forward_named_refusals():
     assert lib.moe_fp4_workspace_size(ctypes.byref(_weights(E=0)), 4, 2) == 0
 
 
+def test_selftest_refusals():
+    lib = L.load()
+    assert lib.fp4_selftest_wait_timeout(None, 1000, None) == 1
+    assert lib.fp4_selftest_wait_timeout(P, 0, None) == 1
+    assert lib.fp4_selftest_wait_timeout(P, 3_000_000_000, None) == 1
+
+
 def test_linear_named_refusals():
     lib = L.load()
     lin = lambda fmt, T, K, N, ws=P: lib.fp4_linear(fmt, P, T, K, P, P, P, N, P, ws, 1 << 40, None)

@@ -97,3 +97,20 @@ def test_moe_c4_full_prefill_sampled_tokens():
     """The full prefill layer (8192 tokens, 256 experts, hidden 6144, inter 2048, top-8)
     through the auto-selected tensor-core kernels; the oracle checks three tokens."""
     _moe_case(C.MOE_C4, tokens=[0, 8191], prepared=True)
+
+
+# Degenerate routings: one token on one expert, every expert selected (k = E), and a
+# single expert (E = 1, k = 1: the layer is a plain SwiGLU FFN), on both expert kernels
+# and all three formats.
+_EDGE = [
+    ("mxfp4", 1, 8, 1, 1), ("mxfp4", 1, 8, 1, 2), ("mxfp4", 5, 4, 4, 1), ("mxfp4", 5, 4, 4, 2),
+    ("mxfp4", 3, 1, 1, 2), ("nvfp4", 3, 1, 1, 1), ("nvfp4", 6, 4, 4, 1), ("cb4", 2, 1, 1, 1), ("cb4", 4, 4, 4, 1),
+]
+
+
+@pytest.mark.parametrize("fmt,T,E,k,variant", _EDGE, ids=[f"{f}_t{t}_e{e}_k{k}_v{v}" for f, t, e, k, v in _EDGE])
+def test_moe_edge_routings(fmt, T, E, k, variant):
+    from dataclasses import replace
+    base = {"mxfp4": C.MOE_C2, "nvfp4": C.MOE_C3, "cb4": C.MOE_C5}[fmt]
+    cfg = replace(base, name=f"edge_{fmt}_t{T}_e{E}_k{k}", T=T, E=E, H=512, I=256, k=k, zipf_bias=False)
+    _moe_case(cfg, variant=variant)
