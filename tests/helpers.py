@@ -11,7 +11,9 @@ ELEM_A = 2e-2        # per-element bound: |err| <= ELEM_A * (|ref| + 1)
 
 
 def check_tolerance(got, ref, mask_rows=None):
-    """Assert the fixed output gates; returns (rel_fro, max_elem_ratio)."""
+    """Assert the fixed output gates; returns (rel_fro, max_elem_ratio).  When the
+    environment names a file in FP4_PARITY_LOG, each call appends one line: the test id,
+    the relative Frobenius error and the largest per-element error ratio."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if mask_rows is not None:
@@ -19,6 +21,11 @@ def check_tolerance(got, ref, mask_rows=None):
     err = got - ref
     rel = np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300)
     ratio = np.max(np.abs(err) / (ELEM_A * (np.abs(ref) + 1.0))) if err.size else 0.0
+    log = __import__("os").environ.get("FP4_PARITY_LOG")
+    if log:
+        case = __import__("os").environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+        with open(log, "a") as f:
+            f.write(f"{case}\trel_fro={rel:.3e}\tmax_elem_ratio={ratio:.4f}\n")
     assert np.all(np.isfinite(got)), "non-finite output"
     assert rel <= REL_FRO, f"relative Frobenius error {rel:.3e} > {REL_FRO}"
     assert ratio <= 1.0, f"per-element error exceeds {ELEM_A}(|ref|+1) by factor {ratio:.3f}"
