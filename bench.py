@@ -189,6 +189,22 @@ def build_layer(cfg, copies, device):
     return weights, x, wr_t, bias_t, x_bits
 
 
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank timings over all ranks (the slowest replica sets
+    the job's time); identity on one rank."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(work_per_rank, world, ms):
+    """Whole-job rate: the work of every replica over the slowest replica's time."""
+    return work_per_rank * world / (ms * 1e-3)
+
+
 def run_ours(args, cfg, rank, world):
     import torch
     import torch.distributed as dist
@@ -294,10 +310,7 @@ def run_ours(args, cfg, rank, world):
 
     gu_ms = kern["gate_up_ns"] / max(kern["gate_up_launches"], 1) / 1e6
     dn_ms = kern["down_ns"] / max(kern["down_launches"], 1) / 1e6
-    t = torch.tensor([ms_total, e2e_ms, gu_ms, dn_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms, gu_ms, dn_ms = t.tolist()
+    ms_total, e2e_ms, gu_ms, dn_ms = max_over_ranks([ms_total, e2e_ms, gu_ms, dn_ms], world, device)
     kern_ms = {"gate_up": gu_ms, "down": dn_ms, "launches": kern["gate_up_launches"]}
     return dict(ms_per_step=ms_total / args.steps, bytes_step=bytes_step, work_step=work_step, extra_gu=extra_gu,
                 e2e_ms=e2e_ms / args.steps,
@@ -457,7 +470,7 @@ def main():
         pass
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
     unit = work_per_step(cfg, r["counts"])[1]
-    value = r["work_step"] * world / (r["ms_per_step"] * 1e-3)
+    value = job_rate(r["work_step"], world, r["ms_per_step"])
     bank_mb = r["copies"] * per_expert_bytes(cfg)[0] * cfg.E / 1e6
     conf = {"workload": workload, "tokens": cfg.T, "experts": cfg.E, "hidden": cfg.H, "inter": cfg.I,
             "top_k": cfg.k, "format": cfg.fmt, "parallelism": f"replicas{world}",
@@ -479,7 +492,7 @@ def main():
                   else ("f16(codebook)xf16->f32" if cfg.fmt == "cb4" else "f16xe2m1->f32")),
         "data": "synthetic",
         "config": conf,
-        "e2e": {"value": r["work_step"] * world / (r["e2e_ms"] * 1e-3), "unit": unit,
+        "e2e": {"value": job_rate(r["work_step"], world, r["e2e_ms"]), "unit": unit,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "roofline": roofline(cfg, r, hbm_peak, peaks, uses_tensor_cores(cfg, args.variant)),
