@@ -16,7 +16,7 @@
 // tiles are 64 gate rows followed by the 64 up rows of the same intermediate indices;
 // down tiles are 128 output rows.
 //
-// Warp roles of one persistent CTA per SM:
+// Warp roles of a persistent CTA (one per SM; two for decode-sized units of <= 64 columns):
 //   warp 0     producer: TMA of the weight tile (two 64-row boxes, FP4 widened to
 //              16-byte slots, 128-byte swizzle) and of the activation-term tile, and one
 //              bulk copy per scale atom (weights: re-laid once by fp4_mma_scales or per
@@ -53,6 +53,7 @@ struct BsLayout {
   int tmem_cols;
   int xch_off, cnt_off, off_off, pre_off, bar_off;
   int smem_bytes;
+  int ctas_per_sm;   // 2 for narrow units (decode), else 1
 };
 
 struct BsUnit {
@@ -556,9 +557,13 @@ bool bs_layout(int T, int E, BsLayout* L) {
   const int b0 = off;
   off += 8 * (2 * kBsMaxStages + 5) + 8 + 4 * (kBsMaxStages + 2);
   const int fixed = static_cast<int>(align_up(off, 16));
-  int S = (kBsSmemLimit - 1024 - fixed) / L->stage_bytes;
+  // narrow units (few tokens per expert) leave the tensor pipe idle between stages: two
+  // CTAs per SM, each with half the shared memory and TMEM, keep two pipelines in flight
+  L->ctas_per_sm = (L->ncols <= 64) ? 2 : 1;
+  const int smem_limit = (L->ctas_per_sm == 2) ? 112 * 1024 : kBsSmemLimit;
+  int S = (smem_limit - 1024 - fixed) / L->stage_bytes;
   S = std::min(S, kBsMaxStages);
-  while (S > 0 && 2 * L->ncols + kSfCols * S > 512) --S;
+  while (S > 0 && 2 * L->ncols + kSfCols * S > 512 / L->ctas_per_sm) --S;
   if (S < 2) return false;
   L->stages = S;
   const int body = S * L->stage_bytes;
@@ -627,8 +632,8 @@ fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st) {
     FP4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmemLimit));
     configured[which] = true;
   }
-  return launch_pdl(kern, dim3(num_sms()), dim3(kBsThreads), static_cast<size_t>(L.smem_bytes), st, true, mA,
-                    mB, a, L);
+  return launch_pdl(kern, dim3(L.ctas_per_sm * num_sms()), dim3(kBsThreads), static_cast<size_t>(L.smem_bytes), st,
+                    true, mA, mB, a, L);
 }
 
 }  // namespace fp4
