@@ -16,7 +16,8 @@
 // tiles are 64 gate rows followed by the 64 up rows of the same intermediate indices;
 // down tiles are 128 output rows.
 //
-// Warp roles of a persistent CTA (one per SM; two for decode-sized units of <= 64 columns):
+// Warp roles of a persistent CTA (one per SM; two or three for decode-sized units of <= 64
+// or <= 32 columns):
 //   warp 0     producer: TMA of the weight tile (two 64-row boxes, FP4 widened to
 //              16-byte slots, 128-byte swizzle) and of the activation-term tile, and one
 //              bulk copy per scale atom (weights: re-laid once by fp4_mma_scales or per
@@ -31,6 +32,7 @@
 #include <algorithm>
 
 #include "kernels.cuh"
+#include "routing.cuh"
 #include "tcgen05.cuh"
 
 namespace fp4 {
@@ -133,6 +135,60 @@ __device__ __forceinline__ void warp_split2(float v, uint32_t& q1, uint32_t& q2,
   s2 = static_cast<uint32_t>(e2 + 127);
 }
 
+// One 32-element block of token row t (bf16) -> its two E4M3 terms in rows 2 slot and
+// 2 slot + 1 of q, and the two UE8M0 scales into the token group's atoms (row 2i, 2i+1).
+__device__ __forceinline__ void split_block(const uint16_t* __restrict__ x, int t, int slot, int b, int i,
+                                            int64_t gid, int H, uint8_t* __restrict__ q,
+                                            uint8_t* __restrict__ atoms) {
+  const int kb128 = H / 128;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + 32 * b);
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 w = src[j];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii) {
+      v[8 * j + 2 * ii] = __uint_as_float(ws[ii] << 16);
+      v[8 * j + 2 * ii + 1] = __uint_as_float(ws[ii] & 0xFFFF0000u);
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int ii = 0; ii < 32; ++ii) amax = fmaxf(amax, fabsf(v[ii]));
+  const int e1 = e4m3_block_exp(amax);
+  const float inv1 = exp2i(-e1), up1 = exp2i(e1);
+  uint32_t w1[8], w2[8];
+  float ramax = 0.f;
+#pragma unroll
+  for (int ii = 0; ii < 32; ++ii) {
+    float b1;
+    const uint32_t c = e4m3_rn(v[ii] * inv1, b1);
+    if ((ii & 3) == 0) w1[ii >> 2] = 0;
+    w1[ii >> 2] |= c << (8 * (ii & 3));
+    v[ii] -= b1 * up1;
+    ramax = fmaxf(ramax, fabsf(v[ii]));
+  }
+  const int e2 = e4m3_block_exp(ramax);
+  const float inv2 = exp2i(-e2);
+#pragma unroll
+  for (int ii = 0; ii < 32; ++ii) {
+    float b2;
+    const uint32_t c = e4m3_rn(v[ii] * inv2, b2);
+    if ((ii & 3) == 0) w2[ii >> 2] = 0;
+    w2[ii >> 2] |= c << (8 * (ii & 3));
+  }
+  uint4* d1 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot)) * H + 32 * b);
+  uint4* d2 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot) + 1) * H + 32 * b);
+  d1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+  d2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+  d2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+  uint8_t* at = atoms + (gid * kb128 + (b >> 2)) * 1024 + (b & 3);
+  at[sf_row_off2(2 * i)] = static_cast<uint8_t>(e1 + 127);
+  at[sf_row_off2(2 * i + 1)] = static_cast<uint8_t>(e2 + 127);
+}
+
 // x [T][H] bf16 -> slot-ordered two-term MXFP8 rows q [2P][H] E4M3 (rows 2i, 2i + 1 for
 // slot i = token perm[i] / k) and their UE8M0 scales as token-group atoms.  One thread
 // per 32-element block.
@@ -165,7 +221,7 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
   }
   for (int e = threadIdx.x; e <= E; e += blockDim.x) off_s[e] = offsets[e];
   __syncthreads();
-  const int nb = H / 32, kb128 = H / 128;
+  const int nb = H / 32;
   const int64_t total = static_cast<int64_t>(P) * nb;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -178,53 +234,99 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
     const int local = slot - off_s[lo];
     const int grp = local / cap, i = local - grp * cap;
     const int64_t gid = gpre_s[lo] + grp;
-    const int t = perm[slot] / k;
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + 32 * b);
-    float v[32];
+    split_block(x, perm[slot] / k, slot, b, i, gid, H, q, atoms);
+  }
+  pdl_launch_dependents();
+}
+
+// Small routing problems (T k <= 1024 slots, E <= 512) in one launch: every CTA forms the
+// top-k of the logits, the per-expert counts and the stable slot order in shared memory
+// (CTA 0 also stores them for the later kernels: ids, gate weights, counts, offsets,
+// perm, inv), then splits its share of the slots' activation rows like split_x_kernel.
+__global__ void __launch_bounds__(512) route_split_kernel(
+    const float* __restrict__ logits, int T, int E, int k, const uint16_t* __restrict__ x, int H, int cap,
+    int32_t* __restrict__ ids, float* __restrict__ gw, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ q, uint8_t* __restrict__ atoms) {
+  __shared__ int ids_s[kRouteMaxPairs], perm_s[kRouteMaxPairs];
+  __shared__ int cnt[kRouteMaxExperts], off[kRouteMaxExperts + 1], cur[kRouteMaxExperts], gpre[kRouteMaxExperts];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int P = T * k;
+  pdl_wait();
+  for (int t = warp; t < T; t += nw)
+    topk_warp(logits + static_cast<int64_t>(t) * E, E, k, ids_s + t * k,
+              blockIdx.x == 0 ? gw + static_cast<int64_t>(t) * k : nullptr);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    atomicAdd(&cnt[ids_s[p]], 1);
+    if (blockIdx.x == 0) ids[p] = ids_s[p];
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive scans: first slot and first token group of every expert
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int sc = 0, sg = 0;
+    for (int e = e0; e < e1; ++e) {
+      sc += cnt[e];
+      sg += (cnt[e] + cap - 1) / cap;
+    }
+    int ic = sc, ig = sg;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 w = src[j];
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii) {
-        v[8 * j + 2 * ii] = __uint_as_float(ws[ii] << 16);
-        v[8 * j + 2 * ii + 1] = __uint_as_float(ws[ii] & 0xFFFF0000u);
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vc = __shfl_up_sync(0xFFFFFFFFu, ic, o), vg = __shfl_up_sync(0xFFFFFFFFu, ig, o);
+      if (lane >= o) { ic += vc; ig += vg; }
+    }
+    int rc = ic - sc, rg = ig - sg;
+    for (int e = e0; e < e1; ++e) {
+      off[e] = rc;
+      cur[e] = rc;
+      gpre[e] = rg;
+      rc += cnt[e];
+      rg += (cnt[e] + cap - 1) / cap;
+    }
+    if (lane == 31) off[E] = ic;
+    __syncwarp();
+    // stable placement: pairs in ascending order, 32 per round, ranked within the round
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < P; base += 32) {
+      const int p = base + lane;
+      const bool live = p < P;
+      const int e = live ? ids_s[p] : -1 - lane;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      const int rank = __popc(peers & lt);
+      const int slot = live ? cur[e] + rank : 0;
+      __syncwarp();
+      if (live && rank == 0) cur[e] += __popc(peers);
+      __syncwarp();
+      if (live) {
+        perm_s[slot] = p;
+        if (blockIdx.x == 0) {
+          perm[slot] = p;
+          inv[p] = slot;
+        }
       }
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int ii = 0; ii < 32; ++ii) amax = fmaxf(amax, fabsf(v[ii]));
-    const int e1 = e4m3_block_exp(amax);
-    const float inv1 = exp2i(-e1), up1 = exp2i(e1);
-    uint32_t w1[8], w2[8];
-    float ramax = 0.f;
-#pragma unroll
-    for (int ii = 0; ii < 32; ++ii) {
-      float b1;
-      const uint32_t c = e4m3_rn(v[ii] * inv1, b1);
-      if ((ii & 3) == 0) w1[ii >> 2] = 0;
-      w1[ii >> 2] |= c << (8 * (ii & 3));
-      v[ii] -= b1 * up1;
-      ramax = fmaxf(ramax, fabsf(v[ii]));
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      if (e < E) counts[e] = cnt[e];
+      offsets[e] = off[e];
     }
-    const int e2 = e4m3_block_exp(ramax);
-    const float inv2 = exp2i(-e2);
-#pragma unroll
-    for (int ii = 0; ii < 32; ++ii) {
-      float b2;
-      const uint32_t c = e4m3_rn(v[ii] * inv2, b2);
-      if ((ii & 3) == 0) w2[ii >> 2] = 0;
-      w2[ii >> 2] |= c << (8 * (ii & 3));
+  const int nb = H / 32;
+  const int64_t total = static_cast<int64_t>(P) * nb;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int slot = static_cast<int>(idx / nb), b = static_cast<int>(idx % nb);
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= slot) lo = mid; else hi = mid - 1;
     }
-    uint4* d1 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot)) * H + 32 * b);
-    uint4* d2 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot) + 1) * H + 32 * b);
-    d1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-    d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
-    d2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-    d2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
-    uint8_t* at = atoms + (gid * kb128 + (b >> 2)) * 1024 + (b & 3);
-    at[sf_row_off2(2 * i)] = static_cast<uint8_t>(e1 + 127);
-    at[sf_row_off2(2 * i + 1)] = static_cast<uint8_t>(e2 + 127);
+    const int local = slot - off[lo];
+    const int grp = local / cap, i = local - grp * cap;
+    split_block(x, perm_s[slot] / k, slot, b, i, static_cast<int64_t>(gpre[lo]) + grp, H, q, atoms);
   }
   pdl_launch_dependents();
 }
@@ -559,11 +661,13 @@ bool bs_layout(int T, int E, BsLayout* L) {
   const int fixed = static_cast<int>(align_up(off, 16));
   // narrow units (few tokens per expert) leave the tensor pipe idle between stages: two
   // CTAs per SM, each with half the shared memory and TMEM, keep two pipelines in flight
-  L->ctas_per_sm = (L->ncols <= 64) ? 2 : 1;
-  const int smem_limit = (L->ctas_per_sm == 2) ? 112 * 1024 : kBsSmemLimit;
+  L->ctas_per_sm = (L->ncols <= 32) ? 3 : ((L->ncols <= 64) ? 2 : 1);
+  const int smem_limit = (L->ctas_per_sm == 3) ? 74 * 1024 : ((L->ctas_per_sm == 2) ? 112 * 1024 : kBsSmemLimit);
   int S = (smem_limit - 1024 - fixed) / L->stage_bytes;
   S = std::min(S, kBsMaxStages);
-  while (S > 0 && 2 * L->ncols + kSfCols * S > 512 / L->ctas_per_sm) --S;
+  // each CTA's allocation (a power of two) must leave room for the others on the SM
+  const int tmem_share = (L->ctas_per_sm == 3) ? 128 : 512 / L->ctas_per_sm;
+  while (S > 0 && 2 * L->ncols + kSfCols * S > tmem_share) --S;
   if (S < 2) return false;
   L->stages = S;
   const int body = S * L->stage_bytes;
@@ -588,6 +692,16 @@ fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t*
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, num_sms() * 16)));
   return launch_pdl(split_x_kernel, dim3(grid), dim3(256), 0, st, true, x, perm, counts, offsets, E, k, P, H,
                     ntok_cap, q, atoms);
+}
+
+fp4_status launch_route_split(const float* logits, int T, int E, int k, const uint16_t* x, int H, int ntok_cap,
+                              int32_t* ids, float* gw, int32_t* counts, int32_t* offsets, int32_t* perm,
+                              int32_t* inv, uint8_t* q, uint8_t* atoms, cudaStream_t st) {
+  if (T * k > kRouteMaxPairs || E > kRouteMaxExperts) return FP4_ERR_UNSUPPORTED;
+  const int64_t total = static_cast<int64_t>(T) * k * (H / 32);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 511) / 512, num_sms())));
+  return launch_pdl(route_split_kernel, dim3(grid), dim3(512), 0, st, true, logits, T, E, k, x, H, ntok_cap, ids, gw,
+                    counts, offsets, perm, inv, q, atoms);
 }
 
 fp4_status launch_mma_scales(const uint8_t* scales, int64_t rows, int64_t K, int64_t pair, uint8_t* atoms,

@@ -20,7 +20,11 @@ int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
   const bool tc_ok = w->fmt == FP4_MXFP4 && bs_supported(T, w->num_experts, w->hidden, w->inter);
   if (w->kernel_variant == kVarTensor) return kVarTensor;
   if (w->kernel_variant == kVarGemv) return kVarGemv;
-  return (tc_ok && static_cast<int64_t>(T) * k >= 4 * static_cast<int64_t>(w->num_experts)) ? kVarTensor : kVarGemv;
+  // tensor cores when the scale atoms come with the weights, or when the call has enough
+  // tokens per expert to amortise re-laying them in the workspace
+  const bool prepared = w->gu_mma_scales != nullptr && w->dn_mma_scales != nullptr;
+  const bool many = static_cast<int64_t>(T) * k >= 4 * static_cast<int64_t>(w->num_experts);
+  return (tc_ok && (prepared || many)) ? kVarTensor : kVarGemv;
 }
 
 struct MoeWs {
@@ -147,8 +151,10 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   ra.sexp = reinterpret_cast<int*>(ws + L.sexp);
   ra.ctrl = reinterpret_cast<WsControl*>(ws + L.status);
   if (moe_variant(w, T, k) == kVarTensor) {
+    // small routing problems: top-k, permutation and the activation split share a launch
+    const bool fused_split = P <= kRouteMaxPairs && E <= kRouteMaxExperts;
     ra.x16 = nullptr;
-    ra.logits_only = false;
+    ra.logits_only = fused_split;
     ra.pdl_first = true;
     FP4_TRY(launch_route(ra, st));
     uint8_t* xq = ws + L.xq;
@@ -164,8 +170,12 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
       FP4_TRY(launch_mma_scales(w->dn_scales, static_cast<int64_t>(E) * H, I, 0, ws + L.adn, st));
       adn = ws + L.adn;
     }
-    FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, ra.counts, ra.offsets, E, k, P, H, cap, xq,
-                           xs, st));
+    if (fused_split)
+      FP4_TRY(launch_route_split(ra.logits, T, E, k, static_cast<const uint16_t*>(x_bf16), H, cap, ra.ids, ra.gw,
+                                 ra.counts, ra.offsets, ra.perm, ra.inv, xq, xs, st));
+    else
+      FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, ra.counts, ra.offsets, E, k, P, H, cap,
+                             xq, xs, st));
     BsArgs g{};
     g.epi = kEpiSwiglu;
     g.codes = w->gu_codes;

@@ -184,8 +184,9 @@ typedef struct fp4_moe_weights {
   const int32_t* dn_rowptr;
   const int32_t* dn_col;
   const uint16_t* dn_val;
-  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores for MXFP4 when T*k >= 4E,
-   * i.e. four or more tokens per expert on average), 1 = CUDA-core grouped GEMV,
+  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores for MXFP4 when
+   * gu_mma_scales / dn_mma_scales are given, or when T*k >= 4E, i.e. four or more tokens
+   * per expert on average; else the CUDA-core GEMV), 1 = CUDA-core grouped GEMV,
    * 2 = block-scaled tensor-core GEMM (MXFP4 only; FP4_ERR_UNSUPPORTED otherwise).
    * Any other value is FP4_ERR_INVALID_ARG. */
   int32_t kernel_variant;
