@@ -286,8 +286,11 @@ fp4_status fp4_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* st
  * allocating library routine.
  *   - Capacity: moe_fp4_noalloc_capacity() bytes (16 MiB) on every device that loads the
  *     library, held until the process exits.  A call whose moe_fp4_workspace_size(w, T, k)
- *     exceeds it returns FP4_ERR_WORKSPACE and launches nothing (16 MiB covers decode
- *     batches such as 64 tokens x top-8 at hidden 6144, intermediate 2048).
+ *     exceeds it returns FP4_ERR_WORKSPACE and launches nothing.  16 MiB covers decode
+ *     batches such as 64 tokens x top-8 at hidden 6144, intermediate 2048 on the CUDA-core
+ *     expert kernels (14.8 MiB), and 16 tokens x top-8 at hidden 2048, intermediate 768
+ *     on the tensor-core kernels (3.3 MiB with re-laid scale atoms); the tensor-core
+ *     kernels at the larger shape need 36.6 MiB and are refused.
  *   - The first call on a device looks up the buffer's device address and clears its
  *     control block; make that first call before any stream capture on that device.
  *   - All calls on a device share the one buffer and it keeps the previous call's
