@@ -15,7 +15,7 @@ Follows [XFP]:
 * 子字节打包: N = 4 packs 8 indices per 32-bit word; a 128-weight group spans
   16 lanes of such words (LANES_PER_GROUP = 128 / 8).
 
-Readings where the pages are silent or differ from the workload (DESIGN.md):
+Readings where the pages are silent or differ from the workload:
 * The workload fits one 16-entry fp16 codebook per 128-weight group of a row
   (not per channel, not a shared library), with the threshold |w - mu| > 6 sigma
   for the nominal sigma = 0.02 and mu = 0, and stores outliers in CSR per

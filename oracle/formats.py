@@ -17,7 +17,7 @@ Definitions followed:
 * Two 4-bit values per byte ([GATE] "A fused tensor with two dtypes in it");
   the element with the even index takes the low nibble.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 * Rounding to E2M1 and to E4M3 is round-to-nearest, ties to the even
   mantissa; values above the largest finite magnitude saturate; the sign of a
   value that rounds to zero is kept (code 8 is -0).

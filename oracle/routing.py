@@ -6,7 +6,7 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
 trunk plus the top-k of E experts (8 of 288, 8 of 256). The workload's
 router is a top-8 softmax router with an optional per-expert logit bias.
 
-Readings (DESIGN.md): logits = x . W_r^T + bias; the k largest logits are
+Readings: logits = x . W_r^T + bias; the k largest logits are
 selected, ties going to the lower expert index, in descending-logit order;
 gate weights are the softmax over the k selected logits (identical to the
 full softmax renormalised over them). The permutation is a stable sort of
