@@ -106,6 +106,37 @@ def test_forward_named_refusals():
     assert lib.moe_fp4_workspace_size(ctypes.byref(_weights(E=0)), 4, 2) == 0
 
 
+def test_mma_scales_refusals():
+    lib = L.load()
+    ms = lambda rows, k, pair=0, src=P, dst=P: lib.fp4_mma_scales(src, rows, k, pair, dst, None)
+    assert ms(0, 256) == 2
+    assert ms(100, 256) == 5                  # rows not a multiple of 128
+    assert ms(128, 200) == 5                  # k not a multiple of 128
+    assert ms(3 * 96, 256, pair=96) == 5      # I not a multiple of 64
+    assert ms(3 * 128, 256, pair=128) == 5    # rows not a multiple of 2I
+    assert ms(128, 256, pair=-1) == 1
+    assert ms(128, 256, src=None) == 1
+    assert ms(128, 256, dst=ctypes.c_void_p(0x10008)) == 4
+
+
+def test_cb4_pack_refusals():
+    lib = L.load()
+    rp = lambda rows, k, thr=0.12, mu=0.0, w=P, dt=L.FP4_F32: lib.fp4_cb4_row_ptr(w, dt, rows, k, thr, mu, P, None)
+    assert rp(0, 128) == 2
+    assert rp(4, 100) == 4                    # k not a multiple of 128
+    assert rp(1 << 24, 1 << 8) == 3           # rows * k >= 2^31
+    assert rp(4, 128, thr=-1.0) == 1
+    assert rp(4, 128, thr=float("nan")) == 1
+    assert rp(4, 128, mu=float("inf")) == 1
+    assert rp(4, 128, w=None) == 1
+    assert rp(4, 128, dt=7) == 1
+    pk = lambda **kw: lib.fp4_pack_cb4(kw.get("w", P), L.FP4_F32, 4, 128, 0.12, 0.0, kw.get("rp", P),
+                                       kw.get("idx", P), kw.get("cb", P), P, P, None)
+    assert pk(rp=None) == 1
+    assert pk(idx=ctypes.c_void_p(0x10004)) == 4
+    assert pk(cb=None) == 1
+
+
 def test_selftest_refusals():
     lib = L.load()
     assert lib.fp4_selftest_wait_timeout(None, 1000, None) == 1
