@@ -1,5 +1,6 @@
-// Grouped W4A16 GEMV for the decode path: few tokens per expert, so the layer is
-// bound by the weight stream from HBM.
+// Grouped W4A16 GEMV on the CUDA cores for decode-sized calls (few tokens per expert, so
+// the layer is bound by the weight stream from HBM): NVFP4, CB4, the dense linear layer,
+// and MXFP4 when its weights come without the tensor-core scale atoms.
 //
 // Design (B200): persistent CTAs, two or three per SM, walk work units {expert, 64-row weight
 // tile, up to 8 routed tokens}.  One producer warp streams a unit's 4-bit codes with TMA
