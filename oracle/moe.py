@@ -73,6 +73,70 @@ class ExpertBank:
         return h @ self.down(e).T
 
 
+class LazyExpertBank:
+    """Expert bank that quantises an expert the first time it is used.
+
+    ``draw(which, e)`` returns the float32 weights of expert e (which = "gu" -> [2I, H],
+    "dn" -> [H, I]); they are quantised here with this package's own formats (MXFP4,
+    NVFP4 with one tensor scale per expert matrix, or CB4 with ``cb4_threshold`` as
+    the absolute outlier threshold around mu = 0) and dequantised exactly in float64.
+    """
+
+    def __init__(self, fmt, E, H, I, draw, cb4_threshold=None):
+        self.fmt, self.E, self.H, self.I = fmt, E, H, I
+        self.draw = draw
+        self.cb4_threshold = cb4_threshold
+        self._cache = {}
+
+    def packed(self, which, e):
+        key = (which, e)
+        if key not in self._cache:
+            w = self.draw(which, e)
+            if self.fmt == "cb4":
+                self._cache[key] = codebook.cb4_fit(w, self.cb4_threshold)
+            elif self.fmt == "mxfp4":
+                self._cache[key] = formats.mxfp4_quantize(w) + (None,)
+            else:
+                c, s, t = formats.nvfp4_quantize(w[None])
+                self._cache[key] = (c[0], s[0], t[0])
+        return self._cache[key]
+
+    def dequant(self, which, e):
+        if self.fmt == "cb4":
+            fit = self.packed(which, e)
+            n, k2 = fit["idx"].shape
+            return (codebook.cb4_dense(fit["idx"], fit["cb_val"])
+                    + codebook.cb4_sparse(fit["row_ptr"], fit["col"], fit["val"], n, 2 * k2))
+        c, s, t = self.packed(which, e)
+        if self.fmt == "mxfp4":
+            return formats.mxfp4_dequantize(c, s)
+        return formats.nvfp4_dequantize(c, s, t)
+
+    def apply_gate_up(self, e, x):
+        return np.asarray(x, dtype=np.float64) @ self.dequant("gu", e).T
+
+    def apply_down(self, e, h):
+        return np.asarray(h, dtype=np.float64) @ self.dequant("dn", e).T
+
+    def preload(self, which, e, packed):
+        """Install an expert's quantised form made earlier by ``packed`` (e.g. in another
+        process) so that later calls skip quantising it."""
+        self._cache[(which, e)] = packed
+
+    def drop(self, e):
+        """Forget the quantised copies of expert e (bounds memory on full-size layers)."""
+        self._cache.pop(("gu", e), None)
+        self._cache.pop(("dn", e), None)
+
+
+def expert_outputs(bank, e, x_rows, limit: float = 7.0):
+    """One expert on the rows routed to it: o = W_d(e) (silu(min(g, L)) clamp(u, -L, L))
+    with [g; u] = W_gu(e) x, float64 [n, H].  The per-expert body of ``moe_forward``."""
+    gu = bank.apply_gate_up(int(e), np.asarray(x_rows, dtype=np.float64))
+    h = swiglu_clamp(gu[:, :bank.I], gu[:, bank.I:], limit)
+    return bank.apply_down(int(e), h)
+
+
 def moe_forward(x, ids, w, bank: ExpertBank, limit: float = 7.0, tokens=None):
     """Routed-expert MoE layer in float64.
 
@@ -83,19 +147,20 @@ def moe_forward(x, ids, w, bank: ExpertBank, limit: float = 7.0, tokens=None):
     x = np.asarray(x, dtype=np.float64)
     T, k = ids.shape
     tok = np.arange(T) if tokens is None else np.asarray(tokens)
-    I = bank.I
     o = np.zeros((tok.size, k, bank.H), dtype=np.float64)
     sub_ids = ids[tok]
     for e in np.unique(sub_ids):
         ti, jj = np.nonzero(sub_ids == e)
-        xe = x[tok[ti]]
-        gu = bank.apply_gate_up(int(e), xe)
-        h = swiglu_clamp(gu[:, :I], gu[:, I:], limit)
-        o[ti, jj] = bank.apply_down(int(e), h)
-    wsub = np.asarray(w, dtype=np.float64)[tok]
-    y = np.zeros((tok.size, bank.H), dtype=np.float64)
-    for j in range(k):
-        y += wsub[:, j:j + 1] * o[:, j]
+        o[ti, jj] = expert_outputs(bank, e, x[tok[ti]], limit)
+    return combine_slots(np.asarray(w, dtype=np.float64)[tok], o)
+
+
+def combine_slots(w, o):
+    """y_t = sum_{j = 0..k-1} w[t, j] o[t, j] accumulated in j order: w [n, k], o [n, k, H]."""
+    w = np.asarray(w, dtype=np.float64)
+    y = np.zeros((o.shape[0], o.shape[2]), dtype=np.float64)
+    for j in range(o.shape[1]):
+        y += w[:, j:j + 1] * o[:, j]
     return y
 
 

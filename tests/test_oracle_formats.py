@@ -201,3 +201,33 @@ def test_nvfp4_error_smaller_than_mxfp4_on_t4():
     e_mx = F.mxfp4_dequantize(*F.mxfp4_quantize(w)) - w
     e_nv = F.nvfp4_dequantize(*F.nvfp4_quantize(w)) - w
     assert np.linalg.norm(e_nv) < np.linalg.norm(e_mx)
+
+
+def test_nvfp4_op_order_non_power_of_two_tensor_scale(golden):
+    """A hand-worked NVFP4 case (tests/golden/nvfp4_op_order.txt) with a tensor scale that
+    is not a power of two: the oracle's codes follow the stated float32 order, and the
+    two plausible slips (ts = amax/6/448; dividing by the block scale and the tensor
+    scale separately) give a different code on the same value."""
+    g = {k: v for k, v in golden("nvfp4_op_order.txt")}
+    f = lambda h: np.frombuffer(bytes.fromhex(h)[::-1], dtype=np.float32)[0]
+    amax_t, amax_b, v = f(g["amax_t_bits"]), f(g["amax_b_bits"]), f(g["v_bits"])
+    w = np.zeros((2, 16), np.float32)
+    w[0, 0], w[1, 0], w[1, 1] = amax_t, amax_b, v
+    codes, scales, ts = F.nvfp4_quantize(w)
+    assert np.float32(ts).tobytes()[::-1].hex() == g["ts_bits"]
+    assert scales[:, 0].tolist() == [int(g["scale_row0"], 16), int(g["scale_row1"], 16)]
+    c = F.unpack_nibbles(codes)
+    assert int(c[0, 0]) == int(g["code_row0_col0"])
+    assert int(c[1, 0]) == int(g["code_row1_col0"])
+    assert int(c[1, 1]) == int(g["code_row1_col1"])
+    assert not c[:, 2:].any() and not c[0, 1:].any()
+    # the slips, evaluated in float32 with the same element rounding, give the tie code
+    sbv = np.float32(F.e4m3_value(scales[1, 0]))
+    ts_slip = np.float32(np.float32(amax_t / np.float32(6)) / np.float32(448))
+    assert ts_slip != ts
+    six = np.float32(6) * ts_slip
+    sb_slip = F.e4m3_round(np.float64(np.float32(amax_b / six)))
+    q1 = np.float32(v / np.float32(np.float32(F.e4m3_value(sb_slip)) * ts_slip))
+    q2 = np.float32(np.float32(v / sbv) / np.float32(ts))
+    assert int(F.e2m1_round(np.float64(q1))) == int(g["slip_code_row1_col1"])
+    assert int(F.e2m1_round(np.float64(q2))) == int(g["slip_code_row1_col1"])
