@@ -25,8 +25,9 @@ void* g_scratch_ptr[kMaxDevices] = {nullptr};
 // Device address of the scratch buffer on the current device.  The first call on a
 // device looks it up with cudaGetSymbolAddress (the host-side name of a __device__
 // array is only a stand-in and must never be passed to a kernel) and clears the
-// workspace control block once; later calls reuse the cached address.
-fp4_status scratch_for_current_device(void** out) {
+// workspace control block once, on the caller's stream so that it is ordered before
+// the kernels the call launches; later calls reuse the cached address.
+fp4_status scratch_for_current_device(void** out, cudaStream_t st) {
   int dev = 0;
   FP4_TRY_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return FP4_ERR_UNSUPPORTED;
@@ -34,7 +35,7 @@ fp4_status scratch_for_current_device(void** out) {
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     FP4_TRY_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-    FP4_TRY_CUDA(cudaMemset(p, 0, 256));    // control block (status word, timing counters)
+    FP4_TRY_CUDA(cudaMemsetAsync(p, 0, 256, st));   // control block (status word, timing counters)
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -42,6 +43,12 @@ fp4_status scratch_for_current_device(void** out) {
 }
 
 }  // namespace
+
+namespace fp4 {
+// The scratch of the current device (set up on first use), for the library's own
+// entry points that act on it (status word, the bounded-wait self-test).
+fp4_status noalloc_scratch(void** out, cudaStream_t st) { return scratch_for_current_device(out, st); }
+}  // namespace fp4
 
 extern "C" size_t moe_fp4_noalloc_capacity(void) { return kNoAllocScratchBytes; }
 
@@ -55,7 +62,13 @@ extern "C" fp4_status moe_fp4_forward_noalloc(const fp4_moe_weights* w, const vo
   }
   if (need > kNoAllocScratchBytes) return FP4_ERR_WORKSPACE;   // larger than the fixed buffer
   void* scratch = nullptr;
-  FP4_TRY(scratch_for_current_device(&scratch));
+  FP4_TRY(scratch_for_current_device(&scratch, static_cast<cudaStream_t>(stream)));
   return moe_fp4_forward(w, x_bf16, router_w, router_bias, T, k, y_bf16, nullptr, scratch,
                          kNoAllocScratchBytes, stream);
+}
+
+extern "C" fp4_status moe_fp4_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  FP4_TRY(scratch_for_current_device(&scratch, static_cast<cudaStream_t>(stream)));
+  return fp4_workspace_status(scratch, stream);
 }

@@ -92,9 +92,13 @@ def test_forward_named_refusals():
     bad = _weights()
     bad.kernel_variant = 7
     assert fwd(bad) == 1                       # unknown kernel variant
-    nv = _weights(fmt=L.FP4_NVFP4)
-    nv.kernel_variant = 2
-    assert fwd(nv) == 5                        # tensor-core variant is MXFP4 only
+    nv1, nv2 = _weights(fmt=L.FP4_NVFP4), _weights(fmt=L.FP4_NVFP4)
+    nv1.kernel_variant, nv2.kernel_variant = 1, 2
+    # NVFP4 on the tensor cores keeps slot-ordered f16 rows of x in the workspace
+    assert lib.moe_fp4_workspace_size(ctypes.byref(nv2), 4, 2) > lib.moe_fp4_workspace_size(ctypes.byref(nv1), 4, 2)
+    assert lib.moe_fp4_expert_kernels(ctypes.byref(nv2), 4, 2) == 2
+    assert lib.moe_fp4_expert_kernels(ctypes.byref(nv1), 4, 2) == 1
+    assert lib.moe_fp4_expert_kernels(ctypes.byref(_weights(E=0)), 4, 2) == 0
     small_w, big_w = _weights(), _weights()
     small_w.kernel_variant, big_w.kernel_variant = 1, 2
     # the tensor-core variant keeps x and h as two-term E4M3 rows in the workspace
@@ -114,6 +118,18 @@ def test_mma_scales_refusals():
     assert ms(128, 200) == 5                  # k not a multiple of 128
     assert ms(3 * 96, 256, pair=96) == 5      # I not a multiple of 64
     assert ms(3 * 128, 256, pair=128) == 5    # rows not a multiple of 2I
+    assert ms(128, 256, pair=-1) == 1
+    assert ms(128, 256, src=None) == 1
+    assert ms(128, 256, dst=ctypes.c_void_p(0x10008)) == 4
+
+
+def test_nvfp4_mma_scales_refusals():
+    lib = L.load()
+    ms = lambda rows, k, pair=0, src=P, dst=P: lib.fp4_nvfp4_mma_scales(src, rows, k, pair, dst, None)
+    assert ms(0, 256) == 2
+    assert ms(100, 256) == 5                  # rows not a multiple of 128
+    assert ms(128, 96) == 5                   # k not a multiple of 64
+    assert ms(3 * 96, 256, pair=96) == 5      # I not a multiple of 64
     assert ms(128, 256, pair=-1) == 1
     assert ms(128, 256, src=None) == 1
     assert ms(128, 256, dst=ctypes.c_void_p(0x10008)) == 4
@@ -139,7 +155,7 @@ def test_cb4_pack_refusals():
 
 def test_selftest_refusals():
     lib = L.load()
-    assert lib.fp4_selftest_wait_timeout(None, 1000, None) == 1
+    assert lib.fp4_selftest_wait_timeout(None, 0, None) == 1
     assert lib.fp4_selftest_wait_timeout(P, 0, None) == 1
     assert lib.fp4_selftest_wait_timeout(P, 3_000_000_000, None) == 1
 

@@ -1,0 +1,67 @@
+"""The layer is deterministic: the same call twice, a call on another workspace, and
+every replay of a captured CUDA graph give identical y bits.  Work units are handed to
+CTAs from an atomic counter, so which CTA runs a unit varies from call to call; each
+unit owns its output rows and sums its K in a fixed order, and the combine adds the k
+slots of a token in j order, so the bits do not depend on that schedule."""
+import numpy as np
+import pytest
+import torch
+
+from synth import configs as C
+
+from helpers import device_weights, host_small_inputs
+
+pytestmark = pytest.mark.gpu
+
+_CASES = [
+    ("c2_full_gemv", C.MOE_C2, 1, False),
+    ("c2_full_tensor", C.MOE_C2, 2, True),
+    ("c3_small_nvfp4", C.small(C.MOE_C3), 0, False),
+    ("c5_small_cb4", C.small(C.MOE_C5), 0, False),
+    ("c4_small_tensor", C.small(C.MOE_C4), 2, False),
+    ("c4_full_tensor", C.MOE_C4, 0, True),
+    ("c3_small_nvfp4_tensor", C.small(C.MOE_C3), 2, False),
+    ("c3_full_nvfp4_tensor", C.MOE_C3, 2, True),
+    ("c4nv_full_tensor", C.MOE_C4_NV, 0, True),
+]
+
+
+@pytest.mark.parametrize("name,cfg,variant,prepared", _CASES, ids=[c[0] for c in _CASES])
+def test_repeat_and_graph_replay_bit_identical(name, cfg, variant, prepared):
+    from fp4_block_scaled_moe_b200 import api, prepare_mma_scales
+    x_bits, wr, bias = host_small_inputs(cfg)
+    w = device_weights(cfg)
+    w.kernel_variant = variant
+    if prepared:
+        prepare_mma_scales(w)
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    wr_t = torch.from_numpy(wr).cuda()
+    bias_t = None if bias is None else torch.from_numpy(bias).cuda()
+    nbytes = api.moe_fp4_workspace_size(w, cfg.T, cfg.k)
+    ws1 = api.alloc_workspace(nbytes, x.device)
+    ws2 = api.alloc_workspace(nbytes + 4096, x.device)
+    y1 = api.moe_fp4_forward(w, x, wr_t, bias_t, cfg.k, workspace=ws1)
+    y2 = api.moe_fp4_forward(w, x, wr_t, bias_t, cfg.k, workspace=ws1)
+    y3 = api.moe_fp4_forward(w, x, wr_t, bias_t, cfg.k, workspace=ws2)
+    torch.cuda.synchronize()
+    b1 = y1.view(torch.int16)
+    assert torch.equal(b1, y2.view(torch.int16)), "second call differs"
+    assert torch.equal(b1, y3.view(torch.int16)), "call on another workspace differs"
+    assert bool(torch.isfinite(y1.float()).all())
+
+    yg = torch.empty_like(y1)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        api.moe_fp4_forward(w, x, wr_t, bias_t, cfg.k, workspace=ws1, y=yg)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            api.moe_fp4_forward(w, x, wr_t, bias_t, cfg.k, workspace=ws1, y=yg)
+    for _ in range(3):
+        yg.fill_(float("nan"))
+        with torch.cuda.stream(s):
+            g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(b1, yg.view(torch.int16)), "graph replay differs"
+    assert api.fp4_workspace_status(ws1) == "FP4_OK"
+    del g
