@@ -36,6 +36,7 @@ class MoEWeightsC(ctypes.Structure):
         ("dn_cb", _vp), ("dn_rowptr", _vp), ("dn_col", _vp), ("dn_val", _vp),
         ("kernel_variant", _i32),
         ("gu_mma_scales", _vp), ("dn_mma_scales", _vp),
+        ("expert_begin", _i32), ("local_experts", _i32),
     ]
 
 
@@ -57,6 +58,7 @@ SIGNATURES = {
     "fp4_selftest_wait_timeout": (_cint, [_vp, _i64, _vp]),
     "fp4_pack": (_cint, [_cint, _vp, _cint, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "fp4_mma_scales": (_cint, [_vp, _i64, _i64, _i64, _vp, _vp]),
+    "fp4_nvfp4_mma_scales": (_cint, [_vp, _i64, _i64, _i64, _vp, _vp]),
     "fp4_cb4_row_ptr": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp]),
     "fp4_pack_cb4": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp, _vp, _vp, _vp,
                              _vp]),
@@ -65,11 +67,16 @@ SIGNATURES = {
     "moe_fp4_workspace_size": (_sz, [ctypes.POINTER(MoEWeightsC), _i32, _i32]),
     "moe_fp4_forward": (_cint, [ctypes.POINTER(MoEWeightsC), _vp, _vp, _vp, _i32, _i32, _vp,
                                 ctypes.POINTER(RouteOutC), _vp, _sz, _vp]),
+    "moe_fp4_forward_partial": (_cint, [ctypes.POINTER(MoEWeightsC), _vp, _vp, _vp, _i32, _i32, _vp,
+                                        ctypes.POINTER(RouteOutC), _vp, _sz, _vp]),
+    "fp4_f32_to_bf16": (_cint, [_vp, _i64, _vp, _vp]),
     "fp4_linear_workspace_size": (_sz, [_i32, _i64]),
     "fp4_linear": (_cint, [_cint, _vp, _i32, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "fp4_workspace_status": (_cint, [_vp, _vp]),
     "moe_fp4_noalloc_capacity": (_sz, []),
     "moe_fp4_forward_noalloc": (_cint, [ctypes.POINTER(MoEWeightsC), _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
+    "moe_fp4_noalloc_status": (_cint, [_vp]),
+    "moe_fp4_expert_kernels": (_i32, [ctypes.POINTER(MoEWeightsC), _i32, _i32]),
     "fp4_workspace_kernel_stats": (_cint, [_vp, _cint, ctypes.POINTER(KernelStatsC), _vp]),
 }
 

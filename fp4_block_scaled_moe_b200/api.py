@@ -69,10 +69,26 @@ def fp4_mma_scales(scales: torch.Tensor, pair: int = 0) -> torch.Tensor:
     return out
 
 
+def fp4_nvfp4_mma_scales(scales: torch.Tensor, pair: int = 0) -> torch.Tensor:
+    """NVFP4 scales [..., rows, k/16] re-laid as the tensor-core kernels' 512-byte atoms
+    (flat uint8); pair = I for gate_up weights, 0 for down weights."""
+    _need(scales, "scales", torch.uint8)
+    k = scales.shape[-1] * 16
+    rows = scales.numel() // scales.shape[-1]
+    out = torch.empty(scales.numel(), dtype=torch.uint8, device=scales.device)
+    L.check("fp4_nvfp4_mma_scales", L.load().fp4_nvfp4_mma_scales(_ptr(scales), rows, k, pair, _ptr(out),
+                                                                   _stream(scales.device)))
+    return out
+
+
 def prepare_mma_scales(weights: "MoEWeights") -> "MoEWeights":
-    """Attach re-laid gate_up / down scales to MXFP4 weights for the tensor-core kernels."""
-    weights.gu_mma_scales = fp4_mma_scales(weights.gu_scales, pair=weights.I)
-    weights.dn_mma_scales = fp4_mma_scales(weights.dn_scales)
+    """Attach re-laid gate_up / down scales to MXFP4 or NVFP4 weights for the tensor-core
+    kernels (a one-time preparation; without it each call re-lays them)."""
+    relay = fp4_mma_scales if weights.fmt == "mxfp4" else fp4_nvfp4_mma_scales
+    if weights.fmt not in ("mxfp4", "nvfp4"):
+        raise ValueError("tensor-core scale atoms exist for MXFP4 and NVFP4 weights only")
+    weights.gu_mma_scales = relay(weights.gu_scales, pair=weights.I)
+    weights.dn_mma_scales = relay(weights.dn_scales)
     return weights
 
 
@@ -174,6 +190,10 @@ class MoEWeights:
     # tensor-core kernels: scales re-laid by fp4_mma_scales (else re-laid every call)
     gu_mma_scales: torch.Tensor | None = None
     dn_mma_scales: torch.Tensor | None = None
+    # expert parallelism: these tensors hold experts [expert_begin, expert_begin + local_experts)
+    # of the E routed experts (0, 0: all of them)
+    expert_begin: int = 0
+    local_experts: int = 0
 
     def c_struct(self):
         s = L.MoEWeightsC()
@@ -181,6 +201,7 @@ class MoEWeights:
         s.num_experts, s.hidden, s.inter = self.E, self.H, self.I
         s.swiglu_limit = self.swiglu_limit
         s.kernel_variant = self.kernel_variant
+        s.expert_begin, s.local_experts = self.expert_begin, self.local_experts
         for name in ("gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales", "dn_tscale", "gu_cb",
                      "gu_rowptr", "gu_col", "gu_val", "dn_cb", "dn_rowptr", "dn_col", "dn_val", "gu_mma_scales",
                      "dn_mma_scales"):
@@ -192,6 +213,12 @@ class MoEWeights:
 def moe_fp4_workspace_size(weights: MoEWeights, T: int, k: int) -> int:
     s = weights.c_struct()
     return int(L.load().moe_fp4_workspace_size(ctypes.byref(s), T, k))
+
+
+def moe_fp4_expert_kernels(weights: MoEWeights, T: int, k: int) -> int:
+    """Expert kernels the library runs for this call shape: 1 CUDA-core GEMV, 2 tensor cores."""
+    s = weights.c_struct()
+    return int(L.load().moe_fp4_expert_kernels(ctypes.byref(s), T, k))
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
@@ -224,6 +251,43 @@ def moe_fp4_forward(weights: MoEWeights, x, router_w, router_bias, k, workspace=
                                                    T, k, _ptr(y), ctypes.byref(ro) if ro is not None else None,
                                                    _ptr(workspace), workspace.numel(), _stream(x.device)))
     return y
+
+
+def moe_fp4_forward_partial(weights: MoEWeights, x, router_w, router_bias, k, workspace=None, route_out=None,
+                            y_partial=None):
+    """float32 [T, H] sum over the slots routed to this shard's experts (expert parallelism;
+    see moe_fp4_forward_partial in include/fp4moe.h)."""
+    lib = L.load()
+    _need(x, "x", torch.bfloat16)
+    _need(router_w, "router_w", torch.float32)
+    T = x.shape[0]
+    s = weights.c_struct()
+    need = int(lib.moe_fp4_workspace_size(ctypes.byref(s), T, k))
+    if workspace is None:
+        if need == 0:
+            raise L.FP4Error("moe_fp4_workspace_size", 1, "invalid layer arguments")
+        workspace = alloc_workspace(need, x.device)
+    if y_partial is None:
+        y_partial = torch.empty((T, weights.H), dtype=torch.float32, device=x.device)
+    ro = None
+    if route_out is not None:
+        ro = L.RouteOutC()
+        for name in ("logits", "topk_ids", "topk_w", "counts", "offsets", "perm", "inv"):
+            t = route_out.get(name)
+            setattr(ro, name, None if t is None else t.data_ptr())
+    L.check("moe_fp4_forward_partial", lib.moe_fp4_forward_partial(
+        ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(router_bias), T, k, _ptr(y_partial),
+        ctypes.byref(ro) if ro is not None else None, _ptr(workspace), workspace.numel(), _stream(x.device)))
+    return y_partial
+
+
+def fp4_f32_to_bf16(x: torch.Tensor, out=None) -> torch.Tensor:
+    """bf16 copy of a float32 tensor, rounded by the library (nearest even)."""
+    _need(x, "x", torch.float32)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    L.check("fp4_f32_to_bf16", L.load().fp4_f32_to_bf16(_ptr(x), x.numel(), _ptr(out), _stream(x.device)))
+    return out
 
 
 def fp4_linear(x, codes, scales, tensor_scale=None, fmt="mxfp4", workspace=None, y=None):
@@ -280,3 +344,9 @@ def moe_fp4_forward_noalloc(weights: MoEWeights, x, router_w, router_bias, k, y=
     L.check("moe_fp4_forward_noalloc", lib.moe_fp4_forward_noalloc(
         ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(router_bias), T, k, _ptr(y), _stream(x.device)))
     return y
+
+
+def moe_fp4_noalloc_status() -> str:
+    """Status word of the no-alloc scratch on the current device (read and cleared)."""
+    code = L.load().moe_fp4_noalloc_status(_stream())
+    return L.STATUS.get(code, str(code))

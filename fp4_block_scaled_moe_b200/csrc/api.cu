@@ -153,6 +153,19 @@ extern "C" fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_
   return launch_mma_scales(scales, rows, k, pair, out, static_cast<cudaStream_t>(stream));
 }
 
+extern "C" fp4_status fp4_nvfp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, int64_t pair,
+                                           uint8_t* out, void* stream) {
+  int64_t n;
+  FP4_TRY(checked_count({rows, k}, &n));
+  if (pair < 0) return FP4_ERR_INVALID_ARG;
+  if (k % 64 != 0) return FP4_ERR_UNSUPPORTED;
+  if (pair == 0 && rows % 128 != 0) return FP4_ERR_UNSUPPORTED;
+  if (pair > 0 && (pair % 64 != 0 || rows % (2 * pair) != 0)) return FP4_ERR_UNSUPPORTED;
+  if (scales == nullptr || out == nullptr) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(scales) || !aligned16(out)) return FP4_ERR_ALIGNMENT;
+  return launch_nv_scales(scales, rows, k, pair, out, static_cast<cudaStream_t>(stream));
+}
+
 namespace fp4 {
 namespace {
 // One CTA waits on an mbarrier phase that nothing completes; the bounded wait gives up
@@ -171,10 +184,10 @@ __global__ void wait_selftest_kernel(uint32_t* status, unsigned long long limit_
 }  // namespace fp4
 
 extern "C" fp4_status fp4_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream) {
-  if (workspace == nullptr) return FP4_ERR_INVALID_ARG;
   if (limit_ns <= 0 || limit_ns > 2000000000ll) return FP4_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP4_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (workspace == nullptr) FP4_TRY(noalloc_scratch(&workspace, st));   // the no-alloc entry point's scratch
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP4_ERR_ALIGNMENT;
   wait_selftest_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t*>(workspace),
                                          static_cast<unsigned long long>(limit_ns));
   FP4_TRY_CUDA(cudaGetLastError());

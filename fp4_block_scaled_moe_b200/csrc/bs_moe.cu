@@ -53,7 +53,7 @@ struct BsLayout {
   int stage_bytes;
   int stages;
   int tmem_cols;
-  int xch_off, cnt_off, off_off, pre_off, bar_off;
+  int xch_off, cnt_off, off_off, pre_off, gpre_off, bar_off;
   int smem_bytes;
   int ctas_per_sm;   // 2 for narrow units (decode), else 1
 };
@@ -62,8 +62,9 @@ struct BsUnit {
   int e, tile, slot0, ntok, gid;    // gid: token group number across experts
 };
 
-__device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* off, const int* pre, int E,
-                                            int tiles, int cap) {
+// gpre: token-group prefix over all experts (the numbering the activation atoms use).
+__device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* off, const int* pre,
+                                            const int* gpre, int E, int tiles, int cap) {
   int lo = 0, hi = E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -78,7 +79,7 @@ __device__ __forceinline__ BsUnit bs_unit_of(int u, const int* cnt, const int* o
   const int grp = local - un.tile * groups;
   un.slot0 = off[lo] + grp * cap;
   un.ntok = min(cap, n - grp * cap);
-  un.gid = pre[lo] / tiles + grp;
+  un.gid = gpre[lo] + grp;
   return un;
 }
 
@@ -379,6 +380,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   int* cnt = reinterpret_cast<int*>(smem + L.cnt_off);
   int* off = reinterpret_cast<int*>(smem + L.off_off);
   int* pre = reinterpret_cast<int*>(smem + L.pre_off);
+  int* gpre = reinterpret_cast<int*>(smem + L.gpre_off);
   const int E = a.E;
   const int tiles = (kEpi == kEpiSwiglu) ? a.inter / 64 : a.rows_per_expert / 128;
 
@@ -414,27 +416,34 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   for (int e = threadIdx.x; e < E; e += kBsThreads) cnt[e] = a.counts[e];
   __syncthreads();
   if (warp == 0) {
+    // slots, token groups (all experts) and work units (only the experts in [e_begin, e_end))
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-    int sc = 0, su = 0;
+    auto groups = [&](int e) { return (cnt[e] + L.ntok_cap - 1) / L.ntok_cap; };
+    auto units = [&](int e) { return (e >= a.e_begin && e < a.e_end) ? groups(e) * tiles : 0; };
+    int sc = 0, su = 0, sg = 0;
     for (int e = e0; e < e1; ++e) {
       sc += cnt[e];
-      su += (cnt[e] + L.ntok_cap - 1) / L.ntok_cap * tiles;
+      su += units(e);
+      sg += groups(e);
     }
-    int ic = sc, iu = su;
+    int ic = sc, iu = su, ig = sg;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int vc = __shfl_up_sync(0xFFFFFFFFu, ic, o), vu = __shfl_up_sync(0xFFFFFFFFu, iu, o);
-      if (lane >= o) { ic += vc; iu += vu; }
+      const int vg = __shfl_up_sync(0xFFFFFFFFu, ig, o);
+      if (lane >= o) { ic += vc; iu += vu; ig += vg; }
     }
-    int rc = ic - sc, ru = iu - su;
+    int rc = ic - sc, ru = iu - su, rg = ig - sg;
     for (int e = e0; e < e1; ++e) {
       off[e] = rc;
       pre[e] = ru;
+      gpre[e] = rg;
       rc += cnt[e];
-      ru += (cnt[e] + L.ntok_cap - 1) / L.ntok_cap * tiles;
+      ru += units(e);
+      rg += groups(e);
     }
-    if (lane == 31) { off[E] = ic; pre[E] = iu; }
+    if (lane == 31) { off[E] = ic; pre[E] = iu; gpre[E] = ig; }
   }
   __syncthreads();
   const int n_units = pre[E];
@@ -458,12 +467,12 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         ++it;
         break;
       }
-      const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
-      const int64_t rbase = static_cast<int64_t>(un.e) * a.rows_per_expert;
+      const BsUnit un = bs_unit_of(u, cnt, off, pre, gpre, E, tiles, L.ntok_cap);
+      const int64_t rbase = static_cast<int64_t>(un.e - a.e_begin) * a.rows_per_expert;   // local expert
       const int64_t y0 = (kEpi == kEpiSwiglu) ? rbase + un.tile * 64 : rbase + un.tile * 128;
       const int64_t y1 = (kEpi == kEpiSwiglu) ? y0 + a.inter : y0 + 64;
       const int brow0 = 2 * un.slot0;
-      const int64_t tile_g = static_cast<int64_t>(un.e) * tiles + un.tile;      // tile across experts
+      const int64_t tile_g = static_cast<int64_t>(un.e - a.e_begin) * tiles + un.tile;   // tile across experts
       const uint8_t* sa = a.a_atoms + tile_g * nk * 512;
       const uint8_t* sb = a.b_atoms + static_cast<int64_t>(un.gid) * nk * 1024;
       const bool two_b = 2 * un.ntok > 128;
@@ -516,7 +525,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       __syncwarp();
       if (u < 0) break;
       tc::fence_after_sync();
-      const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
+      const BsUnit un = bs_unit_of(u, cnt, off, pre, gpre, E, tiles, L.ntok_cap);
       const uint32_t N = static_cast<uint32_t>((2 * un.ntok + 15) & ~15);
       const uint32_t idesc = tc::idesc_mxf8f6f4(5u, 0u, 128u, N);
       const uint32_t d0 = tmem + static_cast<uint32_t>(buf * L.ncols);
@@ -561,7 +570,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const int u = *reinterpret_cast<volatile int*>(&acc_unit[buf]);
       if (u < 0) break;
       tc::fence_after_sync();
-      const BsUnit un = bs_unit_of(u, cnt, off, pre, E, tiles, L.ntok_cap);
+      const BsUnit un = bs_unit_of(u, cnt, off, pre, gpre, E, tiles, L.ntok_cap);
       const uint32_t d0 =
           tmem + static_cast<uint32_t>(buf * L.ncols) + (static_cast<uint32_t>(32 * q) << 16);
       const int N = (2 * un.ntok + 15) & ~15;
@@ -655,6 +664,8 @@ bool bs_layout(int T, int E, BsLayout* L) {
   off += 4 * (E + 1);
   const int p0 = off;
   off += 4 * (E + 1);
+  const int g0 = off;
+  off += 4 * (E + 1);
   off = static_cast<int>(align_up(off, 16));
   const int b0 = off;
   off += 8 * (2 * kBsMaxStages + 5) + 8 + 4 * (kBsMaxStages + 2);
@@ -675,6 +686,7 @@ bool bs_layout(int T, int E, BsLayout* L) {
   L->cnt_off = body + c0;
   L->off_off = body + o0;
   L->pre_off = body + p0;
+  L->gpre_off = body + g0;
   L->bar_off = body + b0;
   L->smem_bytes = body + fixed + 1024;      // + slack for the 1024-byte alignment of the base
   const int need = 2 * L->ncols + kSfCols * S;

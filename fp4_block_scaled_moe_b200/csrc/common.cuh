@@ -193,6 +193,19 @@ __device__ __forceinline__ void slot_end(KernelSlot* s) {
   }
 }
 
+// Per-call reset of a workspace control block, by threads 0 and 1 of one CTA of the
+// call's first kernel (after its dependency wait): status word, work-unit counters, and
+// the per-launch timing fields of both kernel slots (the accumulated totals are kept).
+__device__ __forceinline__ void ctrl_reset_per_call(WsControl* ctrl) {
+  if (ctrl == nullptr || threadIdx.x >= 2) return;
+  if (threadIdx.x == 0) ctrl->status = 0u;
+  ctrl->unit_next[threadIdx.x] = 0u;
+  KernelSlot* s = &ctrl->slot[threadIdx.x];
+  s->start_min = ~0ull;
+  s->end_max = 0ull;
+  s->done = 0u;
+}
+
 // Programmatic dependent launch: wait for the producer grid's memory / let the next grid start.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {

@@ -79,15 +79,17 @@ struct Unit {
   int e, tile, slot0, ntok;
 };
 
-// Exclusive scans by warp 0 over E experts: off = scan(cnt), pre = scan(units per expert).
-__device__ void scan_experts(const int* cnt, int* off, int* pre, int E, int tiles) {
+// Exclusive scans by warp 0 over E experts: off = scan(cnt), pre = scan(units per expert),
+// where only the experts in [e_lo, e_hi) (those whose weights the call holds) have units.
+__device__ void scan_experts(const int* cnt, int* off, int* pre, int E, int tiles, int e_lo, int e_hi) {
   const int lane = threadIdx.x & 31;
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+  auto units = [&](int e) { return (e >= e_lo && e < e_hi) ? (cnt[e] + kTok - 1) / kTok * tiles : 0; };
   int sc = 0, su = 0;
   for (int e = e0; e < e1; ++e) {
     sc += cnt[e];
-    su += (cnt[e] + kTok - 1) / kTok * tiles;
+    su += units(e);
   }
   int ic = sc, iu = su;
 #pragma unroll
@@ -100,7 +102,7 @@ __device__ void scan_experts(const int* cnt, int* off, int* pre, int E, int tile
     off[e] = rc;
     pre[e] = ru;
     rc += cnt[e];
-    ru += (cnt[e] + kTok - 1) / kTok * tiles;
+    ru += units(e);
   }
   if (lane == 31) {
     off[E] = ic;
@@ -139,7 +141,7 @@ __device__ __forceinline__ Unit unit_static(int u, int tiles, int T) {
 
 template <int kEpi>
 __device__ __forceinline__ int64_t unit_row(const DecodeArgs& a, const Unit& un, int r) {
-  const int64_t base = static_cast<int64_t>(un.e) * a.rows_per_expert;
+  const int64_t base = static_cast<int64_t>(un.e - a.e_begin) * a.rows_per_expert;   // local expert
   if (kEpi == kEpiSwiglu)
     return base + (r < 32 ? un.tile * 32 + r : a.inter + un.tile * 32 + (r - 32));
   return base + static_cast<int64_t>(un.tile) * kRows + r;
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
       }
       __syncthreads();
       if (warp == 0) {
-        scan_experts(cnt, off, pre, E, tiles);
+        scan_experts(cnt, off, pre, E, tiles, a.e_begin, a.e_end);
         __syncwarp();
         // stable placement: pairs in ascending order, 32 per round, ranked within the round
         int* cur = pre + E + 1;                      // [E] cursors
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     } else {
       for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = a.counts[e];
       __syncthreads();
-      if (warp == 0) scan_experts(cnt, off, pre, E, tiles);
+      if (warp == 0) scan_experts(cnt, off, pre, E, tiles, a.e_begin, a.e_end);
       __syncthreads();
     }
     n_units = pre[E];
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     const int u = *reinterpret_cast<volatile int*>(&stage_unit[it % L.stages]);
     if (u < 0) break;                              // sentinel: no more work
     const Unit un = get_unit(u);
-    const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e] : 1.0f;   // used after the K loop
+    const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e - a.e_begin] : 1.0f;   // used after the K loop
     float acc[2][4];
 #pragma unroll
     for (int m = 0; m < 2; ++m)
@@ -677,6 +679,44 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     *reinterpret_cast<uint2*>(y + static_cast<int64_t>(tt) * H + h) = make_uint2(lo, hi);
   }
   pdl_launch_dependents();
+}
+
+// Expert-parallel partial sum: only the slots of this call's experts contribute, fp32 out.
+__global__ void __launch_bounds__(256) combine_partial_kernel(const float* __restrict__ o,
+                                                              const int32_t* __restrict__ inv,
+                                                              const int32_t* __restrict__ ids, int T, int k, int H,
+                                                              int e_begin, int e_end, float* __restrict__ y) {
+  pdl_wait();
+  const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int tt = static_cast<int>(i / (H / 4));
+    const int h = static_cast<int>(i % (H / 4)) * 4;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[tt * k + j];
+      if (e < e_begin || e >= e_end) continue;
+      const float4 v = *reinterpret_cast<const float4*>(o + static_cast<int64_t>(inv[tt * k + j]) * H + h);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    *reinterpret_cast<float4*>(y + static_cast<int64_t>(tt) * H + h) = s;
+  }
+  pdl_launch_dependents();
+}
+
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ in, int64_t n,
+                                                          uint16_t* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(in[i]));
+}
+
+fp4_status launch_f32_to_bf16(const float* in, int64_t n, uint16_t* out, cudaStream_t st) {
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, num_sms() * 8)));
+  f32_to_bf16_kernel<<<grid, 256, 0, st>>>(in, n, out);
+  FP4_TRY_CUDA(cudaGetLastError());
+  note_launch();
+  return FP4_OK;
 }
 
 }  // namespace fp4

@@ -49,9 +49,13 @@ struct RouteArgs {
 
 fp4_status launch_route(const RouteArgs& a, cudaStream_t st);
 
+// The fixed scratch buffer of moe_fp4_forward_noalloc on the current device (no_alloc.cu).
+fp4_status noalloc_scratch(void** out, cudaStream_t st);
+
 // x (bf16 [T, H]) -> f16 with a per-row power-of-two scale exponent (see route.cu).
+// ctrl (optional): the call's workspace control block, reset per call (see ctrl_reset_per_call).
 __global__ void x_to_f16_kernel(const uint16_t* __restrict__ x, int T, int H, __half* __restrict__ x16,
-                                int* __restrict__ sexp);
+                                int* __restrict__ sexp, WsControl* __restrict__ ctrl);
 
 // Grouped decode GEMV (register dequantisation + warp-level MMA), see decode.cu.
 enum DecodeEpi { kEpiSwiglu = 0, kEpiDown = 1, kEpiLinear = 2 };
@@ -78,6 +82,7 @@ struct DecodeArgs {
   int rows_per_expert;           // 2I (swiglu) or H (down) or N (linear)
   int inter;                     // I (swiglu: up rows start at I)
   int E, T, topk;
+  int e_begin, e_end;            // experts whose weights the call holds (codes row 0 = expert e_begin)
   const float* logits;           // kModeRoute: [T, E]
   int32_t* ids;                  // kModeRoute: written by CTA 0
   float* gw;                     // gate weights per pair (written by CTA 0 in kModeRoute)
@@ -103,6 +108,12 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl);
 // y[t, :] = bf16(sum_j o[inv[t k + j], :]) in j order.
 __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv, int T, int k, int H,
                                uint16_t* __restrict__ y);
+// y[t, :] = sum over j with e_begin <= ids[t k + j] < e_end of o[inv[t k + j], :], fp32, j order.
+__global__ void combine_partial_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv,
+                                       const int32_t* __restrict__ ids, int T, int k, int H, int e_begin,
+                                       int e_end, float* __restrict__ y);
+// out[i] = bf16(in[i]) (round to nearest even).
+fp4_status launch_f32_to_bf16(const float* in, int64_t n, uint16_t* out, cudaStream_t st);
 
 
 // Block-scaled tensor-core expert GEMM (MXFP4 weights x two-term MXFP8 activations).
@@ -123,6 +134,7 @@ struct BsArgs {
   int rows_per_expert;
   int inter;                      // I (gate rows, then up rows, per expert)
   int E;
+  int e_begin, e_end;             // experts whose weights the call holds (codes row 0 = expert e_begin)
   int P;                          // routed slots T*k
   int ntok_cap;                   // slots per token group
   const int32_t* counts;
@@ -154,5 +166,44 @@ fp4_status launch_route_split(const float* logits, int T, int E, int k, const ui
                               int32_t* inv, uint8_t* q, uint8_t* atoms, cudaStream_t st);
 fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t* counts, const int32_t* offsets,
                           int E, int k, int P, int H, int ntok_cap, uint8_t* q, uint8_t* atoms, cudaStream_t st);
+
+// NVFP4 expert GEMMs on the tensor cores (kind::f16, weights widened to f16 on chip).
+// Scale atoms: 512 bytes per (tile, 64-K stage) holding the four E4M3 block scales of each
+// of the tile's 128 rows at byte 4 r; atom (tile, k / 64) at (tile * (K / 64) + k / 64) * 512,
+// tiles as for the MXFP4 kernels (gate_up: 64 gate rows + the matching 64 up rows).
+struct NvArgs {
+  int epi;                        // kEpiSwiglu or kEpiDown
+  const uint8_t* codes;           // [rows_total][K/2] E2M1 pairs
+  const uint8_t* a_atoms;         // the weights' scale atoms
+  const float* tscale;            // [E] per-expert tensor scale
+  int64_t rows_total;
+  int K;
+  int rows_per_expert;
+  int inter;
+  int E;
+  int e_begin, e_end;             // experts whose weights the call holds (codes row 0 = expert e_begin)
+  int P;
+  int ntok_cap;
+  const int32_t* counts;
+  const __half* b_rows;           // activations [P][K] f16, slot order
+  const int* sx;                  // gate_up: power-of-two exponent of each slot's row
+  float limit;
+  __half* h_out;                  // gate_up out: h [P][I] f16, slot order
+  const float* gw;                // down: gate weights by pair
+  const int32_t* perm;
+  float* o_out;                   // down out: [P][ldo] fp32, slot order
+  int ldo;
+  uint32_t* status;
+  KernelSlot* slot;
+  uint32_t* unit_next;
+};
+int nv_ntok_cap(int T, int E);
+bool nv_supported(int T, int E, int H, int I);
+fp4_status launch_nv(const NvArgs& a, int T, cudaStream_t st);
+fp4_status launch_nv_scales(const uint8_t* scales, int64_t rows, int64_t K, int64_t pair, uint8_t* atoms,
+                            cudaStream_t st);
+// xs[i] = f16(x[perm[i] / k] 2^-sx[i]) for the P routed slots, sx as x_to_f16_kernel picks it.
+fp4_status launch_gather_x16(const uint16_t* x, const int32_t* perm, int k, int P, int H, __half* xs, int* sx,
+                             cudaStream_t st);
 
 }  // namespace fp4

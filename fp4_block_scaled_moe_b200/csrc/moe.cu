@@ -16,8 +16,20 @@ constexpr size_t kAlign = 256;
 enum Variant { kVarGemv = 1, kVarTensor = 2 };
 
 // Which expert-GEMM kernels a call runs (the arguments are already validated).
+// Experts whose weights the call holds: [expert_begin, expert_begin + local_experts), or
+// all E when local_experts is 0.
+int64_t local_count(const fp4_moe_weights* w) {
+  return w->local_experts == 0 ? w->num_experts : w->local_experts;
+}
+
+bool tensor_supported(const fp4_moe_weights* w, int32_t T) {
+  if (w->fmt == FP4_MXFP4) return bs_supported(T, w->num_experts, w->hidden, w->inter);
+  if (w->fmt == FP4_NVFP4) return nv_supported(T, w->num_experts, w->hidden, w->inter);
+  return false;
+}
+
 int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
-  const bool tc_ok = w->fmt == FP4_MXFP4 && bs_supported(T, w->num_experts, w->hidden, w->inter);
+  const bool tc_ok = tensor_supported(w, T);
   if (w->kernel_variant == kVarTensor) return kVarTensor;
   if (w->kernel_variant == kVarGemv) return kVarGemv;
   // tensor cores when the scale atoms come with the weights, or when the call has enough
@@ -31,9 +43,41 @@ struct MoeWs {
   size_t status, logits, ids, gw, counts, offsets, perm, inv, sexp, x16, h, o, xq, xs, hq, hs, agu, adn, total;
 };
 
+// NVFP4 on the tensor cores: f16 activation rows in slot order and their exponents,
+// h as f16, and the weights' scale atoms unless the caller has them.
+bool moe_ws_layout_nv(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
+  const int64_t E = w->num_experts, H = w->hidden, I = w->inter;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  *L = MoeWs{};
+  L->status = take(sizeof(WsControl));
+  L->logits = take(sizeof(float) * T * E);
+  L->ids = take(sizeof(int32_t) * P);
+  L->gw = take(sizeof(float) * P);
+  L->counts = take(sizeof(int32_t) * E);
+  L->offsets = take(sizeof(int32_t) * (E + 1));
+  L->perm = take(sizeof(int32_t) * P);
+  L->inv = take(sizeof(int32_t) * P);
+  L->sexp = take(sizeof(int32_t) * P);                 // per-slot exponents of xs
+  L->xs = take(sizeof(uint16_t) * P * H);
+  L->h = take(sizeof(uint16_t) * P * I);
+  L->o = take(sizeof(float) * P * H);
+  const int64_t El = local_count(w);
+  L->agu = take(w->gu_mma_scales == nullptr ? El * 2 * I * (H / 16) : 0);
+  L->adn = take(w->dn_mma_scales == nullptr ? El * H * (I / 16) : 0);
+  L->total = off;
+  return true;
+}
+
 bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   const int64_t E = w->num_experts, H = w->hidden, I = w->inter;
   const bool tensor = moe_variant(w, T, k) == kVarTensor;
+  if (tensor && w->fmt == FP4_NVFP4) return moe_ws_layout_nv(w, T, k, L);
   const int64_t P = static_cast<int64_t>(T) * k;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -60,8 +104,9 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
   L->xs = take(tensor ? bs_group_atom_bytes(static_cast<int>(P), static_cast<int>(E), cap, static_cast<int>(H)) : 0);
   L->hq = take(tensor ? 2 * P * I : 0);
   L->hs = take(tensor ? bs_group_atom_bytes(static_cast<int>(P), static_cast<int>(E), cap, static_cast<int>(I)) : 0);
-  L->agu = take(tensor && w->gu_mma_scales == nullptr ? E * 2 * I * (H / 32) : 0);
-  L->adn = take(tensor && w->dn_mma_scales == nullptr ? E * H * (I / 32) : 0);
+  const int64_t El = local_count(w);
+  L->agu = take(tensor && w->gu_mma_scales == nullptr ? El * 2 * I * (H / 32) : 0);
+  L->adn = take(tensor && w->dn_mma_scales == nullptr ? El * H * (I / 32) : 0);
   L->total = off;
   return true;
 }
@@ -81,6 +126,9 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (!mul_ok(P, H * 4, &tmp) || !mul_ok(static_cast<int64_t>(T) * E, 4, &tmp)) return FP4_ERR_SHAPE_OVERFLOW;
   if (E * 2 * I >= (int64_t(1) << 31) || E * H >= (int64_t(1) << 31)) return FP4_ERR_SHAPE_OVERFLOW;
   if (k > E || k > 32 || E > 1024) return FP4_ERR_INVALID_ARG;
+  if (w->local_experts < 0 || w->expert_begin < 0 || (w->local_experts == 0 && w->expert_begin != 0) ||
+      static_cast<int64_t>(w->expert_begin) + w->local_experts > E)
+    return FP4_ERR_INVALID_ARG;
   const int B = (w->fmt == FP4_MXFP4) ? 32 : (w->fmt == FP4_NVFP4 ? 16 : 128);
   if (H % B != 0 || I % B != 0) return FP4_ERR_ALIGNMENT;
   if (H % 256 != 0 || I % 256 != 0) return FP4_ERR_UNSUPPORTED;
@@ -97,8 +145,7 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (!w->gu_codes || !w->gu_scales || !w->dn_codes || !w->dn_scales) return FP4_ERR_INVALID_ARG;
   if (w->fmt == FP4_NVFP4 && (!w->gu_tscale || !w->dn_tscale)) return FP4_ERR_INVALID_ARG;
   if (w->kernel_variant < 0 || w->kernel_variant > 2) return FP4_ERR_INVALID_ARG;
-  if (w->kernel_variant == kVarTensor && !(w->fmt == FP4_MXFP4 && bs_supported(T, E, H, I)))
-    return FP4_ERR_UNSUPPORTED;
+  if (w->kernel_variant == kVarTensor && !tensor_supported(w, T)) return FP4_ERR_UNSUPPORTED;
   if (!aligned16(w->gu_codes) || !aligned16(w->gu_scales) || !aligned16(w->dn_codes) || !aligned16(w->dn_scales))
     return FP4_ERR_ALIGNMENT;
   if (!aligned16(w->gu_mma_scales) || !aligned16(w->dn_mma_scales)) return FP4_ERR_ALIGNMENT;
@@ -117,13 +164,34 @@ extern "C" size_t moe_fp4_workspace_size(const fp4_moe_weights* w, int32_t T, in
   return L.total;
 }
 
-extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
-                                      const float* router_bias, int32_t T, int32_t k, void* y_bf16,
-                                      const fp4_route_out* route, void* workspace, size_t ws_bytes,
-                                      void* stream) {
+extern "C" int32_t moe_fp4_expert_kernels(const fp4_moe_weights* w, int32_t T, int32_t k) {
+  if (check_moe(w, T, k) != FP4_OK) return 0;
+  return moe_variant(w, T, k);
+}
+
+namespace fp4 {
+namespace {
+
+// The layer's last step: y = bf16(sum_j o) (full expert set), or the fp32 sum over the
+// slots of the call's experts (expert-parallel partial sum).
+fp4_status launch_combine(const float* o, const int32_t* inv, const int32_t* ids, int T, int k, int H, int e0,
+                          int e1, void* y_bf16, float* y_partial, cudaStream_t st) {
+  const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
+  const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, num_sms() * 8));
+  if (y_partial != nullptr)
+    return launch_pdl(combine_partial_kernel, dim3(grid), dim3(256), 0, st, true, o, inv, ids, T, k, H, e0, e1,
+                      y_partial);
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, true, o, inv, T, k, H,
+                    static_cast<uint16_t*>(y_bf16));
+}
+
+fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
+                            const float* router_bias, int32_t T, int32_t k, void* y_bf16, float* y_partial,
+                            const fp4_route_out* route, void* workspace, size_t ws_bytes, void* stream) {
   FP4_TRY(check_moe(w, T, k));
-  if (!x_bf16 || !router_w || !y_bf16) return FP4_ERR_INVALID_ARG;
-  if (!aligned16(x_bf16) || !aligned16(router_w) || !aligned16(y_bf16)) return FP4_ERR_ALIGNMENT;
+  void* y_out = y_partial ? static_cast<void*>(y_partial) : y_bf16;
+  if (!x_bf16 || !router_w || !y_out) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(router_w) || !aligned16(y_out)) return FP4_ERR_ALIGNMENT;
   MoeWs L;
   moe_ws_layout(w, T, k, &L);
   if (workspace == nullptr || ws_bytes < L.total) return FP4_ERR_WORKSPACE;
@@ -132,6 +200,8 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int E = w->num_experts, H = w->hidden, I = w->inter;
   const int P = T * k;
+  const int El = static_cast<int>(local_count(w));
+  const int e0 = w->expert_begin, e1 = w->expert_begin + El;
 
   auto pick = [](auto* user, void* fallback) { return user ? user : reinterpret_cast<decltype(user)>(fallback); };
   const fp4_route_out none = {};
@@ -150,6 +220,68 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   ra.x16 = reinterpret_cast<__half*>(ws + L.x16);
   ra.sexp = reinterpret_cast<int*>(ws + L.sexp);
   ra.ctrl = reinterpret_cast<WsControl*>(ws + L.status);
+  if (moe_variant(w, T, k) == kVarTensor && w->fmt == FP4_NVFP4) {
+    // router (logits, top-k, permutation), then the slot-ordered f16 activation rows
+    ra.x16 = nullptr;
+    ra.logits_only = false;
+    ra.pdl_first = true;
+    FP4_TRY(launch_route(ra, st));
+    __half* xs = reinterpret_cast<__half*>(ws + L.xs);
+    int* sx = reinterpret_cast<int*>(ws + L.sexp);
+    FP4_TRY(launch_gather_x16(static_cast<const uint16_t*>(x_bf16), ra.perm, k, P, H, xs, sx, st));
+    const uint8_t* agu = w->gu_mma_scales;
+    const uint8_t* adn = w->dn_mma_scales;
+    if (agu == nullptr) {
+      FP4_TRY(launch_nv_scales(w->gu_scales, static_cast<int64_t>(El) * 2 * I, H, I, ws + L.agu, st));
+      agu = ws + L.agu;
+    }
+    if (adn == nullptr) {
+      FP4_TRY(launch_nv_scales(w->dn_scales, static_cast<int64_t>(El) * H, I, 0, ws + L.adn, st));
+      adn = ws + L.adn;
+    }
+    NvArgs g{};
+    g.epi = kEpiSwiglu;
+    g.codes = w->gu_codes;
+    g.a_atoms = agu;
+    g.tscale = w->gu_tscale;
+    g.rows_total = static_cast<int64_t>(El) * 2 * I;
+    g.K = H;
+    g.rows_per_expert = 2 * I;
+    g.inter = I;
+    g.E = E;
+    g.e_begin = e0;
+    g.e_end = e1;
+    g.P = P;
+    g.ntok_cap = nv_ntok_cap(T, E);
+    g.counts = ra.counts;
+    g.b_rows = xs;
+    g.sx = sx;
+    g.limit = w->swiglu_limit;
+    g.h_out = reinterpret_cast<__half*>(ws + L.h);
+    g.status = &ra.ctrl->status;
+    g.slot = &ra.ctrl->slot[0];
+    g.unit_next = &ra.ctrl->unit_next[0];
+    FP4_TRY(launch_nv(g, T, st));
+    NvArgs d = g;
+    d.epi = kEpiDown;
+    d.codes = w->dn_codes;
+    d.a_atoms = adn;
+    d.tscale = w->dn_tscale;
+    d.rows_total = static_cast<int64_t>(El) * H;
+    d.K = I;
+    d.rows_per_expert = H;
+    d.b_rows = g.h_out;
+    d.sx = nullptr;
+    d.h_out = nullptr;
+    d.gw = ra.gw;
+    d.perm = ra.perm;
+    d.o_out = reinterpret_cast<float*>(ws + L.o);
+    d.ldo = H;
+    d.slot = &ra.ctrl->slot[1];
+    d.unit_next = &ra.ctrl->unit_next[1];
+    FP4_TRY(launch_nv(d, T, st));
+    return launch_combine(d.o_out, ra.inv, ra.ids, T, k, H, e0, e1, y_bf16, y_partial, st);
+  }
   if (moe_variant(w, T, k) == kVarTensor) {
     // small routing problems: top-k, permutation and the activation split share a launch
     const bool fused_split = P <= kRouteMaxPairs && E <= kRouteMaxExperts;
@@ -163,11 +295,11 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     const uint8_t* agu = w->gu_mma_scales;
     const uint8_t* adn = w->dn_mma_scales;
     if (agu == nullptr) {
-      FP4_TRY(launch_mma_scales(w->gu_scales, static_cast<int64_t>(E) * 2 * I, H, I, ws + L.agu, st));
+      FP4_TRY(launch_mma_scales(w->gu_scales, static_cast<int64_t>(El) * 2 * I, H, I, ws + L.agu, st));
       agu = ws + L.agu;
     }
     if (adn == nullptr) {
-      FP4_TRY(launch_mma_scales(w->dn_scales, static_cast<int64_t>(E) * H, I, 0, ws + L.adn, st));
+      FP4_TRY(launch_mma_scales(w->dn_scales, static_cast<int64_t>(El) * H, I, 0, ws + L.adn, st));
       adn = ws + L.adn;
     }
     if (fused_split)
@@ -181,11 +313,13 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     g.codes = w->gu_codes;
     g.a_atoms = agu;
     g.ntok_cap = cap;
-    g.rows_total = static_cast<int64_t>(E) * 2 * I;
+    g.rows_total = static_cast<int64_t>(El) * 2 * I;
     g.K = H;
     g.rows_per_expert = 2 * I;
     g.inter = I;
     g.E = E;
+    g.e_begin = e0;
+    g.e_end = e1;
     g.P = P;
     g.counts = ra.counts;
     g.b_q = xq;
@@ -201,7 +335,7 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     d.epi = kEpiDown;
     d.codes = w->dn_codes;
     d.a_atoms = adn;
-    d.rows_total = static_cast<int64_t>(E) * H;
+    d.rows_total = static_cast<int64_t>(El) * H;
     d.K = I;
     d.rows_per_expert = H;
     d.b_q = g.hq;
@@ -213,10 +347,7 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     d.slot = &ra.ctrl->slot[1];
     d.unit_next = &ra.ctrl->unit_next[1];
     FP4_TRY(launch_bs(d, T, st));
-    const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
-    const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, num_sms() * 8));
-    return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, true, static_cast<const float*>(d.o_out),
-                      static_cast<const int32_t*>(ra.inv), T, k, H, static_cast<uint16_t*>(y_bf16));
+    return launch_combine(d.o_out, ra.inv, ra.ids, T, k, H, e0, e1, y_bf16, y_partial, st);
   }
 
   // small routing problems finish inside the gate_up kernel's prologue
@@ -237,11 +368,13 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     g.sp_col = w->gu_col;
     g.sp_val = w->gu_val;
   }
-  g.rows_total = static_cast<int64_t>(E) * 2 * I;
+  g.rows_total = static_cast<int64_t>(El) * 2 * I;
   g.K = H;
   g.rows_per_expert = 2 * I;
   g.inter = I;
   g.E = E;
+  g.e_begin = e0;
+  g.e_end = e1;
   g.T = T;
   g.topk = k;
   g.logits = ra.logits;
@@ -272,7 +405,7 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
     d.sp_col = w->dn_col;
     d.sp_val = w->dn_val;
   }
-  d.rows_total = static_cast<int64_t>(E) * H;
+  d.rows_total = static_cast<int64_t>(El) * H;
   d.K = I;
   d.rows_per_expert = H;
   d.x16 = g.h_out;
@@ -282,18 +415,41 @@ extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf
   d.unit_next = &ra.ctrl->unit_next[1];
   d.ldo = H;
   FP4_TRY(launch_decode(d, st, true));
+  return launch_combine(d.o_out, ra.inv, ra.ids, T, k, H, e0, e1, y_bf16, y_partial, st);
+}
 
-  const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
-  const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, num_sms() * 8));
-  FP4_TRY(launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, true,
-                     static_cast<const float*>(d.o_out), static_cast<const int32_t*>(ra.inv), T, k, H,
-                     static_cast<uint16_t*>(y_bf16)));
-  return FP4_OK;
+}  // namespace
+}  // namespace fp4
+
+extern "C" fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
+                                      const float* router_bias, int32_t T, int32_t k, void* y_bf16,
+                                      const fp4_route_out* route, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  if (w != nullptr && w->local_experts != 0 && w->local_experts != w->num_experts)
+    return FP4_ERR_INVALID_ARG;        // a part of the experts gives a partial sum: moe_fp4_forward_partial
+  if (y_bf16 == nullptr) return FP4_ERR_INVALID_ARG;
+  return moe_forward_impl(w, x_bf16, router_w, router_bias, T, k, y_bf16, nullptr, route, workspace, ws_bytes,
+                          stream);
+}
+
+extern "C" fp4_status moe_fp4_forward_partial(const fp4_moe_weights* w, const void* x_bf16,
+                                              const float* router_w, const float* router_bias, int32_t T,
+                                              int32_t k, float* y_partial, const fp4_route_out* route,
+                                              void* workspace, size_t ws_bytes, void* stream) {
+  if (y_partial == nullptr) return FP4_ERR_INVALID_ARG;
+  return moe_forward_impl(w, x_bf16, router_w, router_bias, T, k, nullptr, y_partial, route, workspace, ws_bytes,
+                          stream);
+}
+
+extern "C" fp4_status fp4_f32_to_bf16(const float* in, int64_t n, void* out, void* stream) {
+  if (n <= 0) return FP4_ERR_EMPTY_SHAPE;
+  if (in == nullptr || out == nullptr) return FP4_ERR_INVALID_ARG;
+  return launch_f32_to_bf16(in, n, static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream));
 }
 
 extern "C" size_t fp4_linear_workspace_size(int32_t T, int64_t K) {
   if (T <= 0 || K <= 0) return 0;
-  return align_up(256, kAlign) + align_up(sizeof(int32_t) * T, kAlign) +
+  return align_up(sizeof(WsControl), kAlign) + align_up(sizeof(int32_t) * T, kAlign) +
          align_up(sizeof(uint16_t) * static_cast<size_t>(T) * static_cast<size_t>(K), kAlign);
 }
 
@@ -315,12 +471,14 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   if (workspace == nullptr || ws_bytes < need) return FP4_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return FP4_ERR_ALIGNMENT;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  int* sexp = reinterpret_cast<int*>(ws + 256);
-  __half* x16 = reinterpret_cast<__half*>(ws + 256 + align_up(sizeof(int32_t) * T, kAlign));
+  WsControl* ctrl = reinterpret_cast<WsControl*>(ws);
+  const size_t ctrl_bytes = align_up(sizeof(WsControl), kAlign);
+  int* sexp = reinterpret_cast<int*>(ws + ctrl_bytes);
+  __half* x16 = reinterpret_cast<__half*>(ws + ctrl_bytes + align_up(sizeof(int32_t) * T, kAlign));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, true,
-                     static_cast<const uint16_t*>(x_bf16), static_cast<int>(T), static_cast<int>(K), x16, sexp));
+                     static_cast<const uint16_t*>(x_bf16), static_cast<int>(T), static_cast<int>(K), x16, sexp,
+                     ctrl));
   DecodeArgs a{};
   a.fmt = fmt;
   a.epi = kEpiLinear;
@@ -333,10 +491,13 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   a.K = static_cast<int>(K);
   a.rows_per_expert = static_cast<int>(N);
   a.static_tiles = static_cast<int>(N / 64);
+  a.e_begin = 0;
+  a.e_end = 1;
   a.x16 = x16;
   a.sexp = sexp;
   a.y_out = static_cast<uint16_t*>(y_bf16);
   a.ldo = static_cast<int>(N);
-  a.status = status;
+  a.status = &ctrl->status;
+  a.slot = &ctrl->slot[0];
   return launch_decode(a, st, true);
 }

@@ -52,11 +52,31 @@ __device__ void x_row_to_f16(const uint16_t* __restrict__ xrow, int H, __half* _
 }
 
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restrict__ x, int T, int H,
-                                                       __half* __restrict__ x16, int* __restrict__ sexp) {
+                                                       __half* __restrict__ x16, int* __restrict__ sexp,
+                                                       WsControl* __restrict__ ctrl) {
   pdl_wait();
+  if (blockIdx.x == 0) ctrl_reset_per_call(ctrl);
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row < T) x_row_to_f16(x + static_cast<int64_t>(row) * H, H, x16 + static_cast<int64_t>(row) * H, sexp + row);
   pdl_launch_dependents();
+}
+
+// Routed slots in slot order as f16 rows with their own power-of-two scale (one warp per
+// slot): the activation operand of the NVFP4 tensor-core expert kernels.
+__global__ void __launch_bounds__(256) gather_x16_kernel(const uint16_t* __restrict__ x,
+                                                         const int32_t* __restrict__ perm, int k, int P, int H,
+                                                         __half* __restrict__ xs, int* __restrict__ sx) {
+  pdl_wait();
+  const int warps = gridDim.x * 8;
+  for (int i = blockIdx.x * 8 + (threadIdx.x >> 5); i < P; i += warps)
+    x_row_to_f16(x + static_cast<int64_t>(perm[i] / k) * H, H, xs + static_cast<int64_t>(i) * H, sx + i);
+  pdl_launch_dependents();
+}
+
+fp4_status launch_gather_x16(const uint16_t* x, const int32_t* perm, int k, int P, int H, __half* xs, int* sx,
+                             cudaStream_t st) {
+  const int grid = std::max(1, std::min((P + 7) / 8, num_sms() * 8));
+  return launch_pdl(gather_x16_kernel, dim3(grid), dim3(256), 0, st, true, x, perm, k, P, H, xs, sx);
 }
 
 // ---------------------------------------------------------------------------------
@@ -468,7 +488,7 @@ fp4_status launch_route(const RouteArgs& a, cudaStream_t st) {
                        a.logits, a.x16, a.sexp, a.ctrl));
   } else if (a.x16 != nullptr) {
     FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((a.T + 7) / 8), dim3(256), 0, st, a.pdl_first,
-                       static_cast<const uint16_t*>(a.x), a.T, a.H, a.x16, a.sexp));
+                       static_cast<const uint16_t*>(a.x), a.T, a.H, a.x16, a.sexp, a.ctrl));
   }
   if (a.logits_only) return FP4_OK;
   const float* lg = a.logits_in ? a.logits_in : a.logits;

@@ -1,6 +1,6 @@
 // sm_100a tensor-core primitives: TMEM allocation, shared-memory matrix descriptors,
-// block-scaled tcgen05.mma (kind::mxf8f6f4), scale-factor copies into TMEM, and TMEM
-// loads.  Inline PTX only; the descriptor bit layouts follow the PTX ISA for sm_100
+// block-scaled tcgen05.mma (kind::mxf8f6f4), 16-bit tcgen05.mma (kind::f16), scale-factor
+// copies into TMEM, and TMEM loads.  Inline PTX only; the descriptor bit layouts follow the PTX ISA for sm_100
 // (the same fields CUTLASS's UMMA descriptors describe).
 #pragma once
 
@@ -76,6 +76,29 @@ __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, u
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// ---- instruction descriptor: kind::f16 -----------------------------------------------
+// D float32; A and B both f16 (ab_fmt 0) or both bf16 (1), both K-major; M = 128, N a
+// multiple of 16 in [16, 256].
+__host__ __device__ __forceinline__ uint32_t idesc_f16(uint32_t M, uint32_t N, uint32_t ab_fmt = 0u) {
+  uint32_t d = 0;
+  d |= 1u << 4;           // D format F32
+  d |= ab_fmt << 7;       // A format
+  d |= ab_fmt << 10;      // B format
+  d |= (N >> 3) << 17;
+  d |= (M >> 4) << 24;
+  return d;
+}
+
+// D[tmem] (+)= A[smem] x B[smem]^T, K = 16 (16-bit operands).
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

@@ -18,9 +18,13 @@
  *
  * Conventions for every entry point:
  *   - Pointers are device pointers unless stated; the caller allocates and owns
- *     every buffer, including workspaces.  The library allocates no device memory.
+ *     every buffer, including workspaces.  The library allocates no device memory,
+ *     with one exception: the fixed 16 MiB module buffer (a __device__ array held on
+ *     every device that loads the library) that moe_fp4_forward_noalloc uses as scratch.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
- *     legacy default stream).  Only fp4_workspace_status synchronises.
+ *     legacy default stream).  Only the status and statistics readers
+ *     (fp4_workspace_status, moe_fp4_noalloc_status, fp4_workspace_kernel_stats)
+ *     synchronise.
  *   - Shapes are checked before any launch with checked 64-bit arithmetic: a zero
  *     dimension returns FP4_ERR_EMPTY_SHAPE, a width, element count, byte size or
  *     index that overflows returns FP4_ERR_SHAPE_OVERFLOW ("TensorFold" pull request
@@ -184,16 +188,25 @@ typedef struct fp4_moe_weights {
   const int32_t* dn_rowptr;
   const int32_t* dn_col;
   const uint16_t* dn_val;
-  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores for MXFP4 when
+  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores for MXFP4 and NVFP4 when
    * gu_mma_scales / dn_mma_scales are given, or when T*k >= 4E, i.e. four or more tokens
    * per expert on average; else the CUDA-core GEMV), 1 = CUDA-core grouped GEMV,
-   * 2 = block-scaled tensor-core GEMM (MXFP4 only; FP4_ERR_UNSUPPORTED otherwise).
+   * 2 = tensor-core GEMM (MXFP4: block-scaled kind::mxf8f6f4; NVFP4: weights widened to
+   * f16 on chip, kind::f16; FP4_ERR_UNSUPPORTED for CB4 or unsupported shapes).
    * Any other value is FP4_ERR_INVALID_ARG. */
   int32_t kernel_variant;
   /* Tensor-core variant only (may be NULL): the gate_up / down scales re-laid by
-   * fp4_mma_scales.  When NULL, each call re-lays them into the workspace. */
+   * fp4_mma_scales (MXFP4) or fp4_nvfp4_mma_scales (NVFP4).  When NULL, each call re-lays
+   * them into the workspace. */
   const uint8_t* gu_mma_scales;
   const uint8_t* dn_mma_scales;
+  /* Expert parallelism: the weight tensors hold experts [expert_begin, expert_begin +
+   * local_experts) of the E routed experts (their first dimension is local_experts; the
+   * router still covers all E).  local_experts = 0 (with expert_begin = 0) means all E.
+   * moe_fp4_forward needs all E; moe_fp4_forward_partial takes any range.  A range
+   * outside [0, E] is FP4_ERR_INVALID_ARG. */
+  int32_t expert_begin;
+  int32_t local_experts;
 } fp4_moe_weights;
 
 /*
@@ -210,6 +223,19 @@ typedef struct fp4_moe_weights {
  */
 fp4_status fp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, int64_t pair, uint8_t* out, void* stream);
 
+/*
+ * fp4_nvfp4_mma_scales: NVFP4 scales [rows, k/16] (E4M3, row-major, as fp4_pack writes
+ * them) re-laid for the tensor-core NVFP4 expert kernels: one 512-byte atom per tile of
+ * 128 rows and 64 k, atom (tile, k/64) at (tile * (k/64) + k/64) * 512, the four block
+ * scales of tile row r at bytes 4r .. 4r+3 (block order).  Tiles as in fp4_mma_scales
+ * (pair = 0: 128 consecutive rows, rows % 128 == 0; pair = I > 0: 64 gate rows then the
+ * matching 64 up rows of each expert with 2I rows, I % 64 == 0).  k % 64 == 0.
+ * out: rows * k / 16 bytes.  FP4_ERR_UNSUPPORTED on other shapes; pointers 16-byte
+ * aligned.  No counterpart in the pages: a layout of this library's MMA kernels.
+ */
+fp4_status fp4_nvfp4_mma_scales(const uint8_t* scales, int64_t rows, int64_t k, int64_t pair, uint8_t* out,
+                                void* stream);
+
 /* Optional copies of the routing results of a forward call (each pointer may be NULL). */
 typedef struct fp4_route_out {
   float* logits;     /* [T, E] */
@@ -225,6 +251,11 @@ typedef struct fp4_route_out {
  * (0 when the arguments are invalid). */
 size_t moe_fp4_workspace_size(const fp4_moe_weights* w, int32_t T, int32_t k);
 
+/* The expert-GEMM kernels moe_fp4_forward runs for these weights, T tokens and top-k
+ * (resolving kernel_variant 0): 1 = CUDA-core grouped GEMV, 2 = tensor-core GEMM;
+ * 0 when the arguments are invalid.  Host only, launches nothing. */
+int32_t moe_fp4_expert_kernels(const fp4_moe_weights* w, int32_t T, int32_t k);
+
 /*
  * moe_fp4_forward: the routed-expert MoE layer.
  *   route (as moe_route) -> for every routed pair (t, j), e = topk_ids[t, j]:
@@ -236,10 +267,10 @@ size_t moe_fp4_workspace_size(const fp4_moe_weights* w, int32_t T, int32_t k);
  * route: optional host struct of device pointers receiving the routing results.
  * Accuracy: float32 accumulation of exactly dequantised weights; against a float64
  * evaluation of the same definition, rel. Frobenius error <= 5e-3 and per-element
- * |err| <= 2e-2 (|ref| + 1).  The tensor-core variant (MXFP4) feeds x and h to the
+ * |err| <= 2e-2 (|ref| + 1).  The MXFP4 tensor-core variant feeds x and h to the
  * MMA as two E4M3 terms per value with a power-of-two scale per 32 (residual about
- * 2^-8 of each value); the CUDA-core variant feeds them as float16 with a per-row
- * power-of-two scale.
+ * 2^-8 of each value); the NVFP4 tensor-core variant and the CUDA-core variant feed
+ * them as float16, x with a power-of-two scale per row (h unscaled).
  */
 fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
                            const float* router_bias, int32_t T, int32_t k, void* y_bf16,
@@ -247,10 +278,32 @@ fp4_status moe_fp4_forward(const fp4_moe_weights* w, const void* x_bf16, const f
                            void* stream);
 
 /*
+ * moe_fp4_forward_partial: one rank's share of an expert-parallel MoE layer.  The experts
+ * are split over ranks, each holding a contiguous range of them (expert_begin,
+ * local_experts); every rank routes all T tokens over all E experts and computes
+ *   y_partial[t, :] = sum over j with expert_begin <= e_tj < expert_begin + local_experts
+ *                     of topk_w[t, j] * o_{t, j}        (float32, j order)
+ * so that the layer output is bf16(sum over ranks of y_partial): the ranks' partial sums
+ * are exchanged with an all-reduce (the expert-parallel placement of "GLM-5.3-Flash-MXFP4",
+ * sections "Serving performance against AMD" and "Serving uplift versus the official FP8
+ * checkpoint": TP4/EP4), and fp4_f32_to_bf16 rounds the sum.  y_partial [T, H] float32;
+ * other arguments, workspace and errors as moe_fp4_forward.
+ */
+fp4_status moe_fp4_forward_partial(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
+                                   const float* router_bias, int32_t T, int32_t k, float* y_partial,
+                                   const fp4_route_out* route, void* workspace, size_t ws_bytes, void* stream);
+
+/* out[i] = bf16(in[i]), round to nearest even, for n float32 values (device pointers).
+ * The last step of an expert-parallel layer after its partial sums are reduced. */
+fp4_status fp4_f32_to_bf16(const float* in, int64_t n, void* out, void* stream);
+
+/*
  * fp4_linear: dense W4A16 layer y [T, N] = bf16(x [T, K] . W^T), W [N, K] in MXFP4 or
  * NVFP4 (codes [N, K/2], scales [N, K/B], tensor_scale [1] for NVFP4, else NULL).
  * 4-bit weights read with bf16 activations ("TensorFold" pull request #1050,
- * W4A16_NVFP4).  workspace: at least fp4_linear_workspace_size(T, K) bytes.
+ * W4A16_NVFP4).  workspace: at least fp4_linear_workspace_size(T, K) bytes, 256-byte
+ * aligned; its first 256 bytes are a control block like moe_fp4_forward's, read by
+ * fp4_workspace_status and by fp4_workspace_kernel_stats (gate_up_* = the linear kernel).
  */
 size_t fp4_linear_workspace_size(int32_t T, int64_t K);
 fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K, const uint8_t* codes,
@@ -269,9 +322,10 @@ fp4_status fp4_workspace_status(const void* workspace, void* stream);
  * waits without faulting the GPU.  Launches one kernel that waits on a shared-memory
  * barrier phase nothing completes; after limit_ns (1 .. 2e9) of device time the wait
  * gives up, sets the timeout bit in the status word of `workspace` (a workspace of
- * moe_fp4_forward, 256-byte aligned) and the kernel returns.  fp4_workspace_status then
- * reports FP4_ERR_TIMEOUT and clears the word; the context stays usable.  No
- * counterpart in the pages.
+ * moe_fp4_forward, 256-byte aligned; NULL = the scratch of moe_fp4_forward_noalloc on
+ * the current device) and the kernel returns.  fp4_workspace_status (for NULL:
+ * moe_fp4_noalloc_status) then reports FP4_ERR_TIMEOUT and clears the word; the context
+ * stays usable.  No counterpart in the pages.
  */
 fp4_status fp4_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
 
@@ -297,10 +351,17 @@ fp4_status fp4_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* st
  *     contents (each call rewrites everything it reads).  Calls that overlap on the GPU
  *     -- on two streams, or from two host threads -- race on it: serialise them.
  *   - Arguments, accuracy and errors otherwise as moe_fp4_forward (no routing outputs).
+ *   - A bounded device wait that gives up records FP4_ERR_TIMEOUT in the buffer's status
+ *     word, as for a workspace; read it with moe_fp4_noalloc_status.  Each call clears
+ *     the word when it starts, so read it after the call it should report on.
+ * moe_fp4_noalloc_status: synchronise `stream`, then return the status word of the
+ * current device's buffer (FP4_OK or FP4_ERR_TIMEOUT) and clear it, as
+ * fp4_workspace_status does for a caller's workspace.
  */
 size_t moe_fp4_noalloc_capacity(void);
 fp4_status moe_fp4_forward_noalloc(const fp4_moe_weights* w, const void* x_bf16, const float* router_w,
                                    const float* router_bias, int32_t T, int32_t k, void* y_bf16, void* stream);
+fp4_status moe_fp4_noalloc_status(void* stream);
 
 /*
  * Per-kernel device time of the grouped expert kernels, accumulated in the workspace

@@ -63,12 +63,24 @@ MOE_C4 = MoEConfig("moe_mxfp4_prefill_e256_h6144_i2048_k8_t8192", "mxfp4", T=819
 MOE_C5 = MoEConfig("moe_cb4_decode_e64_h2048_i768_k8_t16", "cb4", T=16, E=64, H=2048, I=768, k=8,
                    outliers=(0.00394, 6.0, 49.0))
 
-FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5)}
+# NVFP4 on the prefill shape: the prefill layer's dimensions, router and weight
+# distribution with the NVFP4 format (E4M3 scale per 16 and a float32 scale per expert
+# matrix) -- the format x phase pairing the benchmark configurations leave open.
+MOE_C4_NV = MoEConfig("moe_nvfp4_prefill_e256_h6144_i2048_k8_t8192", "nvfp4", T=8192, E=256, H=6144,
+                      I=2048, k=8)
+
+FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5, MOE_C4_NV)}
 # The prefill layer at a quarter of the experts and tokens (same per-expert load, same
 # tile shapes; 1.3 GB of weights): the size used for full hardware-counter captures.
 MOE_C4_PROFILE = MoEConfig("moe_mxfp4_prefill_e64_h6144_i2048_k8_t2048", "mxfp4", T=2048, E=64, H=6144,
                            I=2048, k=8)
-PROFILE = {MOE_C4_PROFILE.name: MOE_C4_PROFILE}
+# The NVFP4 decode layer and the NVFP4 prefill layer at a quarter of the experts (and of
+# the tokens for prefill): 1.36 GB of weights, the sizes used for hardware-counter captures.
+MOE_C3_PROFILE = MoEConfig("moe_nvfp4_decode_e64_h6144_i2048_k8_t16_zipf", "nvfp4", T=16, E=64, H=6144, I=2048,
+                           k=8, zipf_bias=True, outliers=(0.003, 10.0, 49.0))
+MOE_C4NV_PROFILE = MoEConfig("moe_nvfp4_prefill_e64_h6144_i2048_k8_t2048", "nvfp4", T=2048, E=64, H=6144,
+                             I=2048, k=8)
+PROFILE = {c.name: c for c in (MOE_C4_PROFILE, MOE_C3_PROFILE, MOE_C4NV_PROFILE)}
 
 
 def small(cfg):
@@ -80,3 +92,15 @@ def small(cfg):
     if cfg.T > 1000:  # prefill-shaped: many tokens per expert
         return replace(cfg, name=cfg.name + "_small", T=300, E=8, H=512, I=256, k=2)
     return replace(cfg, name=cfg.name + "_small", T=9, E=16, H=768, I=512, k=4)
+
+
+def expert_rows(cfg, which, e):
+    """float32 weights of expert e drawn on the host: which = 'gu' -> [2I, H] (gate rows
+    then up rows), 'dn' -> [H, I].  The same draws the device generator makes for the
+    fused [E, rows, K] tensors."""
+    from . import draws
+    if which == "gu":
+        return draws.expert_weights(cfg.seed, TID_GATE_UP, (cfg.E, 2 * cfg.I, cfg.H), start_row=e * 2 * cfg.I,
+                                    rows=2 * cfg.I, sigma=cfg.sigma, outliers=cfg.outliers)
+    return draws.expert_weights(cfg.seed, TID_DOWN, (cfg.E, cfg.H, cfg.I), start_row=e * cfg.H, rows=cfg.H,
+                                sigma=cfg.sigma, outliers=cfg.outliers)
