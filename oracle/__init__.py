@@ -33,4 +33,4 @@ Sources, cited by page title and section:
 Parity pins (tests/test_oracle_*.py) tie every function here to facts the
 pages or mathematics fix; see each module's docstring for which.
 """
-from . import formats, codebook, routing, moe  # noqa: F401
+from . import formats, codebook, routing, moe, v2a  # noqa: F401
