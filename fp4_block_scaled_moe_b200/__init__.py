@@ -13,7 +13,9 @@ from .api import (  # noqa: F401
     fp4_nvfp4_mma_scales,
     fp4_pack,
     fp4_pack_cb4,
+    fp4_pack_v2a,
     fp4_unpack,
+    fp4_unpack_v2a,
     fp4_workspace_kernel_stats,
     fp4_workspace_status,
     moe_fp4_forward,

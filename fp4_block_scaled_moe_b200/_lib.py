@@ -11,9 +11,9 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfp4moe.so")
 
-FP4_MXFP4, FP4_NVFP4, FP4_CB4 = 1, 2, 3
+FP4_MXFP4, FP4_NVFP4, FP4_CB4, FP4_V2A = 1, 2, 3, 4
 FP4_F32, FP4_BF16 = 0, 1
-FORMATS = {"mxfp4": FP4_MXFP4, "nvfp4": FP4_NVFP4, "cb4": FP4_CB4}
+FORMATS = {"mxfp4": FP4_MXFP4, "nvfp4": FP4_NVFP4, "cb4": FP4_CB4, "v2a": FP4_V2A}
 BLOCK = {FP4_MXFP4: 32, FP4_NVFP4: 16}
 
 STATUS = {
@@ -62,6 +62,10 @@ SIGNATURES = {
     "fp4_cb4_row_ptr": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp]),
     "fp4_pack_cb4": (_cint, [_vp, _cint, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp, _vp, _vp, _vp, _vp,
                              _vp]),
+    "fp4_pack_v2a_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
+    "fp4_pack_v2a": (_cint, [_vp, _cint, _i64, _i64, _i64, _i32, ctypes.c_double, ctypes.c_double, _vp, _vp, _vp,
+                             _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fp4_unpack_v2a": (_cint, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp]),
     "fp4_unpack": (_cint, [_cint, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _cint, _vp]),
     "moe_route": (_cint, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_fp4_workspace_size": (_sz, [ctypes.POINTER(MoEWeightsC), _i32, _i32]),

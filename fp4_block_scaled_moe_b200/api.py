@@ -116,6 +116,46 @@ def fp4_pack_cb4(w: torch.Tensor, threshold: float, mu: float = 0.0):
     return {"idx": idx, "cb": cb, "row_ptr": row_ptr, "col": col[:nnz], "val": val[:nnz]}
 
 
+def fp4_pack_v2a(w: torch.Tensor, n_bits: int, threshold: float, mu: float = 0.0):
+    """V2a pack of w [rows, k] or [batch, rows, k] (float32 or bf16), one 32-codebook
+    library per matrix: returns dict(codes, groups, lib, row_ptr, col, val) (see
+    fp4_pack_v2a in include/fp4moe.h); groups are int64 records [batch * rows, k / 128]."""
+    lib_ = L.load()
+    _need(w, "w")
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("w must be float32 or bfloat16")
+    w3 = w.reshape(-1, w.shape[-2], w.shape[-1]) if w.dim() >= 2 else w
+    batch, rows, k = w3.shape
+    dt = L.FP4_F32 if w.dtype == torch.float32 else L.FP4_BF16
+    dev = w.device
+    R = batch * rows
+    row_ptr = torch.empty(R + 1, dtype=torch.int32, device=dev)
+    L.check("fp4_cb4_row_ptr", lib_.fp4_cb4_row_ptr(_ptr(w3), dt, R, k, float(threshold), float(mu), _ptr(row_ptr),
+                                                    _stream(dev)))
+    nnz = int(row_ptr[-1].item())
+    codes = torch.empty((R, k * n_bits // 8), dtype=torch.uint8, device=dev)
+    groups = torch.empty((R, k // 128), dtype=torch.int64, device=dev)
+    lib = torch.empty((batch, 32, 1 << n_bits), dtype=torch.int16, device=dev)
+    col = torch.empty(max(nnz, 1), dtype=torch.int32, device=dev)
+    val = torch.empty(max(nnz, 1), dtype=torch.int16, device=dev)
+    need = int(lib_.fp4_pack_v2a_workspace_size(batch, rows, k, n_bits))
+    if need == 0:
+        raise L.FP4Error("fp4_pack_v2a_workspace_size", 5, "unsupported shape")
+    ws = alloc_workspace(need, dev)
+    L.check("fp4_pack_v2a", lib_.fp4_pack_v2a(_ptr(w3), dt, batch, rows, k, n_bits, float(threshold), float(mu),
+                                              _ptr(row_ptr), _ptr(codes), _ptr(groups), _ptr(lib), _ptr(col),
+                                              _ptr(val), _ptr(ws), ws.numel(), _stream(dev)))
+    return {"codes": codes, "groups": groups, "lib": lib, "row_ptr": row_ptr, "col": col[:nnz], "val": val[:nnz]}
+
+
+def fp4_unpack_v2a(codes, groups, lib, batch, rows, k, n_bits):
+    """Dense V2a term as float32 [batch, rows, k] (exact fp16 values)."""
+    out = torch.empty((batch, rows, k), dtype=torch.float32, device=codes.device)
+    L.check("fp4_unpack_v2a", L.load().fp4_unpack_v2a(_ptr(codes), _ptr(groups), _ptr(lib), batch, rows, k, n_bits,
+                                                      _ptr(out), _stream(codes.device)))
+    return out
+
+
 def fp4_unpack(codes, scales, tensor_scale=None, fmt="mxfp4", out_dtype=torch.float32):
     lib = L.load()
     f = fmt_code(fmt)

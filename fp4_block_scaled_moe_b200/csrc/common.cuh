@@ -67,6 +67,7 @@ fp4_status make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner_by
 // ------------------------------------------------------------------------------------
 
 constexpr uint32_t kStatusTimeout = 1u;   // bit set in the workspace status word
+constexpr int kV2aLibBytes = 32 * 16 * 2;  // a V2a library: 32 codebooks of 16 fp16 entries
 
 // Control block at the start of every workspace (first 256 bytes).
 struct KernelSlot {
@@ -230,6 +231,13 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
   uint32_t h;
   asm("{\n .reg .b16 lo;\n cvt.u16.u32 lo, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}" : "=r"(h) : "r"(w));
   return h;
+}
+
+// a * b + c per f16 half, rounded once (fma)
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {

@@ -181,10 +181,13 @@ template <int kFmt, int kEpi, int kMode, int KC>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a, const Layout L) {
   // stage geometry (must match make_layout)
+  constexpr bool kCb = (kFmt == FP4_CB4 || kFmt == FP4_V2A);      // codebook lookup formats
   constexpr int kB = (kFmt == FP4_MXFP4) ? 32 : 16;
-  constexpr int kScaleRow = (kFmt == FP4_CB4) ? KC / 4 : KC / kB;   // scale (codebook) bytes per row per stage
+  // scale bytes per row per stage (CB4: fp16 codebooks; V2a: 8-byte group records)
+  constexpr int kScaleRow = (kFmt == FP4_CB4) ? KC / 4 : ((kFmt == FP4_V2A) ? KC / 16 : KC / kB);
   constexpr int kScalesOff = kRows * KC / 2;
-  constexpr int kXOff = kScalesOff + kRows * kScaleRow;
+  constexpr int kLibOff = kScalesOff + kRows * kScaleRow;           // V2a: the expert's library (1 KB)
+  constexpr int kXOff = kLibOff + ((kFmt == FP4_V2A) ? kV2aLibBytes : 0);
   constexpr int kXRow = 2 * KC + 64;                 // padded f16 token row
   constexpr int kNq = KC / 128;                      // 32-K regions per warp per stage
   extern __shared__ uint8_t smem_raw[];
@@ -323,8 +326,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
       const int64_t y0 = unit_row<kEpi>(a, un, 0), y1 = unit_row<kEpi>(a, un, 32);
       int xr = 0;
       if (lane < un.ntok) xr = (kEpi == kEpiSwiglu) ? perm_at(un.slot0 + lane) / a.topk : un.slot0 + lane;
-      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2 +
-                                                (kFmt == FP4_CB4 ? kRows * kScaleRow : 0));
+      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2 + (kCb ? kRows * kScaleRow : 0) +
+                                                (kFmt == FP4_V2A ? kV2aLibBytes : 0));
       constexpr int words = kScaleRow / 4;
       for (int c = 0; c < L.nchunks; ++c, ++it) {
         const int s = it % L.stages;
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st_base = sbase + s * L.stage_bytes;
         const int k0 = c * KC;
-        if (kFmt != FP4_CB4) {
+        if (!kCb) {
           for (int w = lane; w < kRows * words; w += 32) {
             const int r = w / words, cw = w - r * words;
             const uint8_t* src = a.scales + unit_row<kEpi>(a, un, r) * (a.K / B) + k0 / B + cw * 4;
@@ -347,10 +350,14 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         __syncwarp();
-        if (kFmt == FP4_CB4)
+        if (kCb)
           for (int r = lane; r < kRows; r += 32)
-            bulk_g2s(st_base + kScalesOff + r * kScaleRow, a.scales + unit_row<kEpi>(a, un, r) * (a.K / 4) + k0 / 4,
+            bulk_g2s(st_base + kScalesOff + r * kScaleRow,
+                     a.scales + unit_row<kEpi>(a, un, r) * (a.K / (KC / kScaleRow)) + k0 / (KC / kScaleRow),
                      static_cast<uint32_t>(kScaleRow), bar_full + 8 * s);
+        if (kFmt == FP4_V2A && lane == 0)
+          bulk_g2s(st_base + kLibOff, a.lib + static_cast<int64_t>(un.e - a.e_begin) * kV2aLibBytes, kV2aLibBytes,
+                   bar_full + 8 * s);
         for (int q = lane; q < 2 * ncb; q += 32) {
           const int rb = q & 1, cb = q >> 1;
           tma_load_2d(st_base + (cb * kRows + rb * 32) * 128, &tmap, k0 / 2 + cb * 128,
@@ -385,7 +392,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
 #pragma unroll
   for (int jj = 0; jj < kNq; ++jj) c_xo[jj] = static_cast<uint32_t>((((jbase & 7) + jj) ^ g) << 4);
   const uint32_t s_off = kScalesOff + rbase * kScaleRow +
-                         (kFmt == FP4_MXFP4 ? jbase : (kFmt == FP4_NVFP4 ? 2 * jbase : (jbase >> 2) * 32));
+                         (kFmt == FP4_MXFP4 ? jbase
+                                            : (kFmt == FP4_NVFP4 ? 2 * jbase : (jbase >> 2) * (kFmt == FP4_CB4 ? 32 : 8)));
   const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
   // per-slot epilogue factors, loaded once so no unit's epilogue waits on global memory
   float* scl_s = reinterpret_cast<float*>(smem + L.scl_off);
@@ -429,9 +437,22 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const uint8_t* sp = stp + s_off + m * 8 * kScaleRow;
-        if (kFmt == FP4_CB4) {
-          const uint4 c0 = *reinterpret_cast<const uint4*>(sp);
-          const uint4 c1 = *reinterpret_cast<const uint4*>(sp + 16);
+        if (kCb) {
+          uint4 c0, c1;
+          if (kFmt == FP4_CB4) {
+            c0 = *reinterpret_cast<const uint4*>(sp);
+            c1 = *reinterpret_cast<const uint4*>(sp + 16);
+          } else {
+            // V2a: the group's entries are fp16(mid + scale * library entry), one rounding each
+            const uint2 rec = *reinterpret_cast<const uint2*>(sp);
+            const uint8_t* lrow = stp + kLibOff + (rec.y & 31u) * 32;
+            const uint4 l0 = *reinterpret_cast<const uint4*>(lrow), l1 = *reinterpret_cast<const uint4*>(lrow + 16);
+            const uint32_t mid2 = __byte_perm(rec.x, 0u, 0x1010), sc2 = __byte_perm(rec.x, 0u, 0x3232);
+            c0 = make_uint4(hfma2(l0.x, sc2, mid2), hfma2(l0.y, sc2, mid2), hfma2(l0.z, sc2, mid2),
+                            hfma2(l0.w, sc2, mid2));
+            c1 = make_uint4(hfma2(l1.x, sc2, mid2), hfma2(l1.y, sc2, mid2), hfma2(l1.z, sc2, mid2),
+                            hfma2(l1.w, sc2, mid2));
+          }
           const uint32_t e[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -458,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
 #pragma unroll
         for (int m = 0; m < 4; ++m) w[m] = *reinterpret_cast<const uint32_t*>(cp + m * 8 * 128);
         uint32_t p[4][4];
-        if (kFmt == FP4_CB4) {
+        if (kCb) {
 #pragma unroll
           for (int m = 0; m < 4; ++m) cb4_lookup8(w[m], tlo[m], thi[m], p[m]);
         } else {
@@ -466,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
           for (int m = 0; m < 4; ++m) e2m1x8_to_f16x8(w[m], p[m][0], p[m][1], p[m][2], p[m][3]);
         }
         const uint4 xq = *reinterpret_cast<const uint4*>(stp + x_off + jj * 64);
-        if (kFmt == FP4_CB4) {
+        if (kCb) {
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt) {
             mma_16816(acc[mt], p[2 * mt][0], p[2 * mt + 1][0], p[2 * mt][1], p[2 * mt + 1][1], xq.x, xq.y);
@@ -534,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     // ---- fused epilogue ----
     // CB4 sparse term of row r against an activation row (same scaling as the MMA input)
     auto sparse = [&](int r, const __half* xrow) -> float {
-      if (kFmt != FP4_CB4 || a.sp_rowptr == nullptr) return 0.f;
+      if (!kCb || a.sp_rowptr == nullptr) return 0.f;
       const int64_t R = unit_row<kEpi>(a, un, r);
       float acc_s = 0.f;
       for (int j = a.sp_rowptr[R]; j < a.sp_rowptr[R + 1]; ++j)
@@ -547,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         const float sc = (L.scl_n > 0) ? ts * scl_s[un.slot0 + i]
                                        : ldexpf(ts, a.sexp[perm_at(un.slot0 + i) / a.topk]);
         const __half* xrow =
-            (kFmt == FP4_CB4) ? a.x16 + static_cast<int64_t>(perm_at(un.slot0 + i) / a.topk) * a.K : nullptr;
+            kCb ? a.x16 + static_cast<int64_t>(perm_at(un.slot0 + i) / a.topk) * a.K : nullptr;
         const float gv = fminf((val(r, i) + sparse(r, xrow)) * sc, a.limit);
         const float uv = fminf(fmaxf((val(32 + r, i) + sparse(32 + r, xrow)) * sc, -a.limit), a.limit);
         const float hv = gv / (1.0f + expf(-gv)) * uv;
@@ -577,14 +598,15 @@ Layout make_layout(int fmt, int K, int E, int P, int P_scl) {
   Layout L{};
   const int B = (fmt == FP4_MXFP4) ? 32 : 16;
   // CB4 stages carry 4 codebook bytes per 16 indices: the smaller stage keeps 5 in flight
-  const int kc = (fmt != FP4_CB4 && K % 512 == 0) ? 512 : ((K % 256 == 0) ? 256 : 0);
+  const bool cb = (fmt == FP4_CB4 || fmt == FP4_V2A);
+  const int kc = (!cb && K % 512 == 0) ? 512 : ((K % 256 == 0) ? 256 : 0);
   if (kc == 0) return L;
   L.kc = kc;
   L.nchunks = K / kc;
-  L.scale_row = (fmt == FP4_CB4) ? kc / 4 : kc / B;
+  L.scale_row = (fmt == FP4_CB4) ? kc / 4 : ((fmt == FP4_V2A) ? kc / 16 : kc / B);
   L.codes_off = 0;
   L.scales_off = kRows * kc / 2;
-  L.x_off = L.scales_off + kRows * L.scale_row;
+  L.x_off = L.scales_off + kRows * L.scale_row + ((fmt == FP4_V2A) ? kV2aLibBytes : 0);
   L.x_row = 2 * kc + 64;
   L.stage_bytes = static_cast<int>(align_up(L.x_off + kTok * L.x_row, 1024));
   const int Eb = static_cast<int>(align_up(sizeof(int) * (E + 1), 16));
@@ -624,7 +646,7 @@ fp4_status launch_kc(const DecodeArgs& a, const Layout& L, const CUtensorMap& ma
 template <int kFmt, int kEpi, int kMode>
 fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
                       bool pdl) {
-  if constexpr (kFmt != FP4_CB4) {
+  if constexpr (kFmt != FP4_CB4 && kFmt != FP4_V2A) {
     if (L.kc == 512) return launch_kc<kFmt, kEpi, kMode, 512>(a, L, map, grid, st, pdl);
   }
   return launch_kc<kFmt, kEpi, kMode, 256>(a, L, map, grid, st, pdl);
@@ -654,6 +676,7 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
   int grid = ctas_per_sm(L.kc) * num_sms();
   if (a.mode == kModeStatic) grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok));
   if (a.fmt == FP4_CB4) return dispatch<FP4_CB4>(a, L, map, grid, st, pdl);
+  if (a.fmt == FP4_V2A) return dispatch<FP4_V2A>(a, L, map, grid, st, pdl);
   return (a.fmt == FP4_NVFP4) ? dispatch<FP4_NVFP4>(a, L, map, grid, st, pdl)
                               : dispatch<FP4_MXFP4>(a, L, map, grid, st, pdl);
 }

@@ -72,7 +72,9 @@ struct DecodeArgs {
   int epi;                       // DecodeEpi
   int mode;                      // DecodeMode
   const uint8_t* codes;          // [rows_total, K/2] (CB4: 4-bit codebook indices)
-  const uint8_t* scales;         // [rows_total, K/B] (CB4: fp16 codebooks [rows_total, K/128, 16])
+  const uint8_t* scales;         // [rows_total, K/B] (CB4: fp16 codebooks [rows_total, K/128, 16];
+                                 //  V2a: 8-byte group records [rows_total, K/128])
+  const uint8_t* lib;            // V2a: libraries [E_local][32][16] fp16
   const int32_t* sp_rowptr;      // CB4 sparse term: CSR over rows_total rows (or null)
   const int32_t* sp_col;
   const uint16_t* sp_val;        // fp16 bits

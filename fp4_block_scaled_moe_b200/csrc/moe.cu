@@ -32,10 +32,13 @@ int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
   const bool tc_ok = tensor_supported(w, T);
   if (w->kernel_variant == kVarTensor) return kVarTensor;
   if (w->kernel_variant == kVarGemv) return kVarGemv;
-  // tensor cores when the scale atoms come with the weights, or when the call has enough
-  // tokens per expert to amortise re-laying them in the workspace
+  // MXFP4: tensor cores when the scale atoms come with the weights, or when the call has
+  // enough tokens per expert to amortise re-laying them in the workspace.  NVFP4: tensor
+  // cores only for the latter (at decode sizes the weight-widening tensor-core kernel
+  // streams slower than the CUDA-core GEMV).
   const bool prepared = w->gu_mma_scales != nullptr && w->dn_mma_scales != nullptr;
   const bool many = static_cast<int64_t>(T) * k >= 4 * static_cast<int64_t>(w->num_experts);
+  if (w->fmt == FP4_NVFP4) return (tc_ok && many) ? kVarTensor : kVarGemv;
   return (tc_ok && (prepared || many)) ? kVarTensor : kVarGemv;
 }
 
@@ -113,7 +116,8 @@ bool moe_ws_layout(const fp4_moe_weights* w, int32_t T, int32_t k, MoeWs* L) {
 
 fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (w == nullptr) return FP4_ERR_INVALID_ARG;
-  if (w->fmt != FP4_MXFP4 && w->fmt != FP4_NVFP4 && w->fmt != FP4_CB4) return FP4_ERR_INVALID_ARG;
+  if (w->fmt != FP4_MXFP4 && w->fmt != FP4_NVFP4 && w->fmt != FP4_CB4 && w->fmt != FP4_V2A)
+    return FP4_ERR_INVALID_ARG;
   int64_t n;
   FP4_TRY(checked_count({w->num_experts, w->hidden, w->inter, T}, &n));
   if (k <= 0) return FP4_ERR_EMPTY_SHAPE;
@@ -129,13 +133,15 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (w->local_experts < 0 || w->expert_begin < 0 || (w->local_experts == 0 && w->expert_begin != 0) ||
       static_cast<int64_t>(w->expert_begin) + w->local_experts > E)
     return FP4_ERR_INVALID_ARG;
-  const int B = (w->fmt == FP4_MXFP4) ? 32 : (w->fmt == FP4_NVFP4 ? 16 : 128);
+  const int B = (w->fmt == FP4_MXFP4) ? 32 : (w->fmt == FP4_NVFP4 ? 16 : 128);   // CB4 / V2a: 128-groups
   if (H % B != 0 || I % B != 0) return FP4_ERR_ALIGNMENT;
   if (H % 256 != 0 || I % 256 != 0) return FP4_ERR_UNSUPPORTED;
   if (!(w->swiglu_limit > 0.f) || !(w->swiglu_limit <= 128.f)) return FP4_ERR_INVALID_ARG;
-  if (w->fmt == FP4_CB4) {
+  if (w->fmt == FP4_CB4 || w->fmt == FP4_V2A) {
     if (!w->gu_codes || !w->gu_cb || !w->dn_codes || !w->dn_cb || !w->gu_rowptr || !w->dn_rowptr)
       return FP4_ERR_INVALID_ARG;
+    if (w->fmt == FP4_V2A && (!w->gu_scales || !w->dn_scales)) return FP4_ERR_INVALID_ARG;
+    if (w->fmt == FP4_V2A && (!aligned16(w->gu_scales) || !aligned16(w->dn_scales))) return FP4_ERR_ALIGNMENT;
     if (!aligned16(w->gu_codes) || !aligned16(w->gu_cb) || !aligned16(w->dn_codes) || !aligned16(w->dn_cb))
       return FP4_ERR_ALIGNMENT;
     if (w->kernel_variant == kVarTensor) return FP4_ERR_UNSUPPORTED;
@@ -362,8 +368,9 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
   g.mode = fused ? kModeRoute : kModeList;
   g.codes = w->gu_codes;
   g.scales = (w->fmt == FP4_CB4) ? reinterpret_cast<const uint8_t*>(w->gu_cb) : w->gu_scales;
+  g.lib = (w->fmt == FP4_V2A) ? reinterpret_cast<const uint8_t*>(w->gu_cb) : nullptr;
   g.tscale = w->gu_tscale;
-  if (w->fmt == FP4_CB4) {
+  if (w->fmt == FP4_CB4 || w->fmt == FP4_V2A) {
     g.sp_rowptr = w->gu_rowptr;
     g.sp_col = w->gu_col;
     g.sp_val = w->gu_val;
@@ -399,8 +406,9 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
   d.mode = kModeList;
   d.codes = w->dn_codes;
   d.scales = (w->fmt == FP4_CB4) ? reinterpret_cast<const uint8_t*>(w->dn_cb) : w->dn_scales;
+  d.lib = (w->fmt == FP4_V2A) ? reinterpret_cast<const uint8_t*>(w->dn_cb) : nullptr;
   d.tscale = w->dn_tscale;
-  if (w->fmt == FP4_CB4) {
+  if (w->fmt == FP4_CB4 || w->fmt == FP4_V2A) {
     d.sp_rowptr = w->dn_rowptr;
     d.sp_col = w->dn_col;
     d.sp_val = w->dn_val;
@@ -456,7 +464,8 @@ extern "C" size_t fp4_linear_workspace_size(int32_t T, int64_t K) {
 extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K,
                                  const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
                                  int64_t N, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
-  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return (fmt == FP4_CB4) ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4)
+    return (fmt == FP4_CB4 || fmt == FP4_V2A) ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
   int64_t n;
   FP4_TRY(checked_count({T, K, N}, &n));
   int64_t tmp;

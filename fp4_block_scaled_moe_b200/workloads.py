@@ -11,7 +11,7 @@ import torch
 
 from synth import configs as C, device as SD
 
-from .api import MoEWeights, fp4_pack, fp4_pack_cb4
+from .api import MoEWeights, fp4_pack, fp4_pack_cb4, fp4_pack_v2a
 
 
 def device_weights_cb4(cfg, device="cuda"):
@@ -30,10 +30,30 @@ def device_weights_cb4(cfg, device="cuda"):
                       dn_cb=dn["cb"], dn_rowptr=dn["row_ptr"], dn_col=dn["col"], dn_val=dn["val"])
 
 
+def device_weights_v2a(cfg, device="cuda"):
+    """V2a weights (4-bit codes, one shared library per expert matrix) drawn and packed
+    on the device with fp4_pack_v2a (one CSR per fused matrix)."""
+    out = {}
+    for which, tid, rows, K in (("gu", C.TID_GATE_UP, 2 * cfg.I, cfg.H), ("dn", C.TID_DOWN, cfg.H, cfg.I)):
+        w = torch.empty((cfg.E * rows, K), dtype=torch.float32, device=device)
+        SD.expert_weights_into(w, cfg.seed, tid, start_row=0, sigma=cfg.sigma, outliers=cfg.outliers)
+        out[which] = fp4_pack_v2a(w.view(cfg.E, rows, K), cfg.v2a_bits, cfg.cb4_threshold_sigma * cfg.sigma)
+        del w
+    gu, dn = out["gu"], out["dn"]
+    return MoEWeights(cfg.fmt, cfg.E, cfg.H, cfg.I, gu["codes"].view(cfg.E, 2 * cfg.I, -1),
+                      gu["groups"].view(torch.uint8).view(cfg.E, 2 * cfg.I, -1),
+                      dn["codes"].view(cfg.E, cfg.H, -1), dn["groups"].view(torch.uint8).view(cfg.E, cfg.H, -1),
+                      None, None, cfg.swiglu_limit,
+                      gu_cb=gu["lib"], gu_rowptr=gu["row_ptr"], gu_col=gu["col"], gu_val=gu["val"],
+                      dn_cb=dn["lib"], dn_rowptr=dn["row_ptr"], dn_col=dn["col"], dn_val=dn["val"])
+
+
 def device_weights(cfg, device="cuda", chunk_elems=1 << 28):
     """Draw every expert's weights of ``cfg`` on the device and pack them there."""
     if cfg.fmt == "cb4":
         return device_weights_cb4(cfg, device)
+    if cfg.fmt == "v2a":
+        return device_weights_v2a(cfg, device)
     B = 32 if cfg.fmt == "mxfp4" else 16
     out = {}
     for which, tid, rows, K in (("gu", C.TID_GATE_UP, 2 * cfg.I, cfg.H), ("dn", C.TID_DOWN, cfg.H, cfg.I)):

@@ -11,6 +11,9 @@
  *   CB4    4-bit indices into a 16-entry fp16 codebook per 128-weight group of a row,
  *          plus a sparse fp16 outlier term in CSR (same page, sections V2, 离群值提取,
  *          Lloyd 迭代, 子字节打包).
+ *   V2A    N-bit codes into one of a matrix's 32 shared fp16 codebooks of 2^N entries,
+ *          chosen per 128-weight group, with an fp16 scale and mid-point per group, plus
+ *          the same sparse outlier term (same page, section V2a：共享码本库).
  * Packing: two 4-bit values per byte, the element with the even index in the low
  * nibble ("The gate that missed by 0.0202 pp", section "A fused tensor with two
  * dtypes in it").  Every tensor is row-major and contiguous:
@@ -63,7 +66,7 @@ typedef enum fp4_status {
   FP4_ERR_TIMEOUT = 8         /* a bounded device-side wait gave up */
 } fp4_status;
 
-typedef enum fp4_format { FP4_MXFP4 = 1, FP4_NVFP4 = 2, FP4_CB4 = 3 } fp4_format;
+typedef enum fp4_format { FP4_MXFP4 = 1, FP4_NVFP4 = 2, FP4_CB4 = 3, FP4_V2A = 4 } fp4_format;
 
 typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
 
@@ -136,6 +139,38 @@ fp4_status fp4_pack_cb4(const void* w, fp4_dtype w_dtype, int64_t rows, int64_t 
                         void* stream);
 
 /*
+ * V2a packing ("XFP：质量地板驱动的自适应码本量化", section V2a：共享码本库, with 离群值提取 and
+ * Lloyd 迭代): w [batch, rows, k] (float32 or bf16, device) holds `batch` matrices; each
+ * gets one library of 32 fp16 codebooks of 2^n_bits entries (n_bits 2 or 4).
+ *   - outliers |w - mu| > threshold leave the bulk (back-filled with mu) for an fp16
+ *     residual CSR over the batch * rows rows; row_ptr [batch * rows + 1] comes from
+ *     fp4_cb4_row_ptr with the same threshold and mu (call it first to size col / val);
+ *   - per 128-group: mid = fp16((max + min) / 2), scale = fp16((max - min) / 2) of the
+ *     bulk, z = (w - mid) / scale (0 when scale is 0);
+ *   - LibFit: a Lloyd codebook per row over its z values (2^n_bits entries started at the
+ *     sorted positions floor((2i + 1) k / 2^(n_bits + 1)), 20 rounds), then Lloyd over the
+ *     rows' codebooks as vectors (32 entries started at the codebooks of span rank
+ *     floor((2i + 1) rows / 64), 20 rounds, squared distance summed in entry order), the
+ *     library rounded to fp16;
+ *   - a group takes the library codebook with the least sum of squared distances to the
+ *     nearest entry (in position order), each weight its nearest entry;
+ *   - reconstruction fp16(mid + scale * entry), rounded once; val = fp16(w - it).
+ * Float64 arithmetic, member means summed in ascending order, ties to the lower index:
+ * deterministic.  Outputs: codes [batch * rows, k * n_bits / 8] (low bits first),
+ * groups [batch * rows, k / 128] 8-byte records (mid fp16 | scale fp16 << 16 | library
+ * index << 32), lib [batch, 32, 2^n_bits] fp16 bits, col / val [nnz] (may be NULL only
+ * when nnz == 0).  workspace: fp4_pack_v2a_workspace_size bytes (256-byte aligned).
+ * Limits: k % 128 == 0 (ALIGNMENT), k <= 4096, 32 <= rows <= 8192 (UNSUPPORTED).
+ * fp4_unpack_v2a: the dense term as float32 (exact fp16 values) [batch, rows, k].
+ */
+size_t fp4_pack_v2a_workspace_size(int64_t batch, int64_t rows, int64_t k, int32_t n_bits);
+fp4_status fp4_pack_v2a(const void* w, fp4_dtype w_dtype, int64_t batch, int64_t rows, int64_t k, int32_t n_bits,
+                        double threshold, double mu, const int32_t* row_ptr, uint8_t* codes, uint64_t* groups,
+                        uint16_t* lib, int32_t* col, uint16_t* val, void* workspace, size_t ws_bytes, void* stream);
+fp4_status fp4_unpack_v2a(const uint8_t* codes, const uint64_t* groups, const uint16_t* lib, int64_t batch,
+                          int64_t rows, int64_t k, int32_t n_bits, float* out, void* stream);
+
+/*
  * moe_route: router of the MoE layer ("The gate that missed by 0.0202 pp", section
  * "A file is a census; a decode step is a sample": each token reads k of E experts).
  *   logits[t, e] = sum_h x[t, h] * router_w[e, h] + router_bias[e]   (float32 accumulate)
@@ -164,6 +199,9 @@ fp4_status moe_route(const void* x_bf16, const float* router_w, const float* rou
  *     [E, rows, K/128, 16] (uint16 bit patterns); the sparse term is one CSR over the
  *     E*rows rows of the fused matrix: *_rowptr [E*rows + 1], *_col [nnz] (column in
  *     the row), *_val [nnz] fp16 bits.  Forward = dense codebook term + sparse term.
+ *   V2A (N = 4 in the layer): *_codes packed 4-bit codes [E, rows, K/2]; *_scales the
+ *     8-byte group records [E, rows, K/128] (fp4_pack_v2a); *_cb the libraries
+ *     [E, 32, 16] fp16 bits (one per expert matrix); the sparse term as for CB4.
  * swiglu_limit: L of h = silu(min(g, L)) * clamp(u, -L, L), finite, 0 < L <= 128.  Experts
  *   apply the model's gated SwiGLU together with its clamp ("GLM-5.3-Flash-MXFP4" model
  *   card, section "Verification compute and EAGLE"); the workload uses L = 7.
@@ -188,9 +226,9 @@ typedef struct fp4_moe_weights {
   const int32_t* dn_rowptr;
   const int32_t* dn_col;
   const uint16_t* dn_val;
-  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores for MXFP4 and NVFP4 when
-   * gu_mma_scales / dn_mma_scales are given, or when T*k >= 4E, i.e. four or more tokens
-   * per expert on average; else the CUDA-core GEMV), 1 = CUDA-core grouped GEMV,
+  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores when T*k >= 4E, i.e. four
+   * or more tokens per expert on average, and for MXFP4 also whenever gu_mma_scales /
+   * dn_mma_scales are given; else the CUDA-core GEMV), 1 = CUDA-core grouped GEMV,
    * 2 = tensor-core GEMM (MXFP4: block-scaled kind::mxf8f6f4; NVFP4: weights widened to
    * f16 on chip, kind::f16; FP4_ERR_UNSUPPORTED for CB4 or unsupported shapes).
    * Any other value is FP4_ERR_INVALID_ARG. */
