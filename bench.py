@@ -52,7 +52,8 @@ from synth import configs as C, draws as D  # noqa: E402
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "FP4 MoE layer: decode HBM GB/s (% of peak); prefill TFLOP/s; tokens/s"
 HEADLINE = C.MOE_C4.name
-ORDER = [C.MOE_C4.name, C.LINEAR_C1.name, C.MOE_C2.name, C.MOE_C3.name, C.MOE_C5.name, C.MOE_C4_NV.name]
+ORDER = [C.MOE_C4.name, C.LINEAR_C1.name, C.MOE_C2.name, C.MOE_C3.name, C.MOE_C5.name, C.MOE_C4_NV.name,
+         C.MOE_C5_V2A.name]
 
 
 def parse(argv=None):
@@ -80,6 +81,8 @@ def per_expert_bytes(cfg):
     dn = cfg.H * cfg.I
     if cfg.fmt == "cb4":
         return (gu + dn) // 2 + (gu + dn) // 4, gu // 2 + gu // 4
+    if cfg.fmt == "v2a":       # 4-bit codes + an 8-byte record per 128 weights + a 1 KB library per matrix
+        return (gu + dn) // 2 + (gu + dn) // 16 + 2 * 1024, gu // 2 + gu // 16 + 1024
     B = 32 if cfg.fmt == "mxfp4" else 16
     b = (gu + dn) // 2 + (gu + dn) // B
     if cfg.fmt == "nvfp4":
@@ -383,7 +386,7 @@ def run_moe(args, cfg, device, world, peaks):
     torch.cuda.synchronize()
     counts = route["counts"].cpu().numpy()
     extra_gu = extra_all = None
-    if cfg.fmt == "cb4":
+    if cfg.fmt in ("cb4", "v2a"):
         extra_gu, extra_all = cb4_extra_bytes(w0)
     work_step, unit = work_per_step(cfg, counts, extra=extra_all)
     graphs, launches = [], 0
@@ -468,6 +471,8 @@ def dtype_label(cfg, tensor):
     """Operand types of the expert MMAs the library ran -> accumulator type."""
     if cfg.fmt == "cb4":
         return "f16(codebook)xf16->f32"
+    if cfg.fmt == "v2a":
+        return "f16(shared-library codebook)xf16->f32"
     if tensor and cfg.fmt == "mxfp4":
         return "e4m3x2xe2m1->f32"
     return "f16xf16(e2m1*e4m3)->f32" if cfg.fmt == "nvfp4" else "f16xe2m1->f32"
@@ -626,7 +631,7 @@ def _quantise_expert(cfg, which, e):
     """Worker: the oracle's quantised form of one expert matrix (untimed preparation)."""
     from oracle import moe as M
     bank = M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
     return bank.packed(which, e)
 
 
@@ -641,7 +646,7 @@ def oracle_pairs(cfg):
     bias = D.zipf_bias(cfg.seed, cfg.E) if cfg.zipf_bias else None
     ids = R.topk(R.router_logits(x0, wr, bias), cfg.k)[0]
     bank = M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
     jobs = [(which, int(e)) for e in ids for which in ("gu", "dn")]
     with cf.ProcessPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1)),
                                 mp_context=mp.get_context("spawn"), initializer=_limit_threads) as pool:
@@ -649,7 +654,7 @@ def oracle_pairs(cfg):
             bank.preload(which, e, packed)
     per, _ = per_expert_bytes(cfg)
     csr = {}
-    if cfg.fmt == "cb4":
+    if cfg.fmt in ("cb4", "v2a"):
         for e in ids:
             csr[int(e)] = sum(6 * int(bank.packed(w, int(e))["row_ptr"][-1]) + 4 * r
                               for w, r in (("gu", 2 * cfg.I), ("dn", cfg.H)))

@@ -15,7 +15,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import formats, codebook, routing
+from . import formats, codebook, routing, v2a
 
 
 def silu(z):
@@ -78,14 +78,16 @@ class LazyExpertBank:
 
     ``draw(which, e)`` returns the float32 weights of expert e (which = "gu" -> [2I, H],
     "dn" -> [H, I]); they are quantised here with this package's own formats (MXFP4,
-    NVFP4 with one tensor scale per expert matrix, or CB4 with ``cb4_threshold`` as
-    the absolute outlier threshold around mu = 0) and dequantised exactly in float64.
+    NVFP4 with one tensor scale per expert matrix, CB4 or V2a (``v2a_bits`` per code,
+    one library per expert matrix) with ``cb4_threshold`` as the absolute outlier
+    threshold around mu = 0) and dequantised exactly in float64.
     """
 
-    def __init__(self, fmt, E, H, I, draw, cb4_threshold=None):
+    def __init__(self, fmt, E, H, I, draw, cb4_threshold=None, v2a_bits=4):
         self.fmt, self.E, self.H, self.I = fmt, E, H, I
         self.draw = draw
         self.cb4_threshold = cb4_threshold
+        self.v2a_bits = v2a_bits
         self._cache = {}
 
     def packed(self, which, e):
@@ -94,6 +96,8 @@ class LazyExpertBank:
             w = self.draw(which, e)
             if self.fmt == "cb4":
                 self._cache[key] = codebook.cb4_fit(w, self.cb4_threshold)
+            elif self.fmt == "v2a":
+                self._cache[key] = v2a.v2a_fit(w, self.v2a_bits, self.cb4_threshold)
             elif self.fmt == "mxfp4":
                 self._cache[key] = formats.mxfp4_quantize(w) + (None,)
             else:
@@ -102,6 +106,8 @@ class LazyExpertBank:
         return self._cache[key]
 
     def dequant(self, which, e):
+        if self.fmt == "v2a":
+            return v2a.v2a_matrix(self.packed(which, e), self.H if which == "gu" else self.I)
         if self.fmt == "cb4":
             fit = self.packed(which, e)
             n, k2 = fit["idx"].shape

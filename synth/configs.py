@@ -44,8 +44,10 @@ class MoEConfig:
     zipf_bias: bool = False
     # planted outliers: (fraction, lo_sigma, hi_sigma) or None
     outliers: tuple | None = None
-    # CB4 only: absolute outlier threshold for the sparse term
+    # CB4 / V2a: absolute outlier threshold for the sparse term (in sigma)
     cb4_threshold_sigma: float = 6.0
+    # V2a: bits per code (N)
+    v2a_bits: int = 4
     swiglu_limit: float = 7.0
     seed: int = SEED
     sigma: float = SIGMA
@@ -69,7 +71,12 @@ MOE_C5 = MoEConfig("moe_cb4_decode_e64_h2048_i768_k8_t16", "cb4", T=16, E=64, H=
 MOE_C4_NV = MoEConfig("moe_nvfp4_prefill_e256_h6144_i2048_k8_t8192", "nvfp4", T=8192, E=256, H=6144,
                       I=2048, k=8)
 
-FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5, MOE_C4_NV)}
+# The V2a shared-library variant of the codebook layer: the CB4 layer's dimensions,
+# weights and outliers, with 4-bit codes into one 32-codebook library per expert matrix.
+MOE_C5_V2A = MoEConfig("moe_v2a4_decode_e64_h2048_i768_k8_t16", "v2a", T=16, E=64, H=2048, I=768, k=8,
+                       outliers=(0.00394, 6.0, 49.0))
+
+FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5, MOE_C4_NV, MOE_C5_V2A)}
 # The prefill layer at a quarter of the experts and tokens (same per-expert load, same
 # tile shapes; 1.3 GB of weights): the size used for full hardware-counter captures.
 MOE_C4_PROFILE = MoEConfig("moe_mxfp4_prefill_e64_h6144_i2048_k8_t2048", "mxfp4", T=2048, E=64, H=6144,
@@ -87,7 +94,7 @@ def small(cfg):
     """A reduced copy of ``cfg`` with the same structure, for exhaustive CPU comparison."""
     if cfg.kind == "linear":
         return replace(cfg, name=cfg.name + "_small", T=5, N=320, K=768)
-    if cfg.fmt == "cb4":
+    if cfg.fmt in ("cb4", "v2a"):
         return replace(cfg, name=cfg.name + "_small", T=7, E=8, H=512, I=256, k=3)
     if cfg.T > 1000:  # prefill-shaped: many tokens per expert
         return replace(cfg, name=cfg.name + "_small", T=300, E=8, H=512, I=256, k=2)

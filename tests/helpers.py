@@ -76,7 +76,7 @@ def oracle_bank(cfg):
     """The oracle's lazily quantised expert bank for a workload (host draws)."""
     from oracle import moe as M
     return M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
 
 
 LazyOracleBank = oracle_bank

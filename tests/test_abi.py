@@ -135,6 +135,24 @@ def test_nvfp4_mma_scales_refusals():
     assert ms(128, 256, dst=ctypes.c_void_p(0x10008)) == 4
 
 
+def test_v2a_pack_refusals():
+    lib = L.load()
+    ws = lambda b, r, k, n: lib.fp4_pack_v2a_workspace_size(b, r, k, n)
+    assert ws(2, 64, 256, 4) > 0 and ws(2, 64, 256, 2) > 0
+    assert ws(2, 64, 256, 3) == 0                   # only 2- and 4-bit codes pack a 128-group evenly
+    assert ws(2, 16, 256, 4) == 0                   # fewer rows than library entries
+    assert ws(2, 64, 200, 4) == 0                   # k not a multiple of 128
+    pk = lambda b, r, k, n, thr=0.12, w=P, wsz=1 << 30: lib.fp4_pack_v2a(
+        w, 0, b, r, k, n, thr, 0.0, P, P, P, P, P, P, P, wsz, None)
+    assert pk(0, 64, 256, 4) == 2
+    assert pk(1, 64, 200, 4) == 4
+    assert pk(1, 64, 256, 3) == 1
+    assert pk(1, 16, 256, 4) == 5
+    assert pk(1, 64, 256, 4, thr=-1.0) == 1
+    assert pk(1, 64, 256, 4, w=PMIS) == 4
+    assert pk(1, 64, 256, 4, wsz=16) == 6
+
+
 def test_cb4_pack_refusals():
     lib = L.load()
     rp = lambda rows, k, thr=0.12, mu=0.0, w=P, dt=L.FP4_F32: lib.fp4_cb4_row_ptr(w, dt, rows, k, thr, mu, P, None)

@@ -96,10 +96,18 @@ def _moe_case(cfg, tokens=None, variant=0, prepared=False, x_scale=1.0, parallel
     return check_tolerance(_y_host(y)[tok], ref)
 
 
-@pytest.mark.parametrize("cfg", [C.small(C.MOE_C2), C.small(C.MOE_C3), C.small(C.MOE_C4), C.small(C.MOE_C5)],
-                         ids=["c2_small", "c3_small", "c4_small_prefill_shape", "c5_small_cb4"])
+@pytest.mark.parametrize("cfg", [C.small(C.MOE_C2), C.small(C.MOE_C3), C.small(C.MOE_C4), C.small(C.MOE_C5),
+                                 C.small(C.MOE_C5_V2A)],
+                         ids=["c2_small", "c3_small", "c4_small_prefill_shape", "c5_small_cb4", "v2a_small"])
 def test_moe_small(cfg):
     _moe_case(cfg)
+
+
+def test_moe_v2a_full_sampled_tokens():
+    """The V2a layer at full size (the CB4 layer's dimensions and outliers, 4-bit codes
+    into one shared 32-codebook library per expert matrix), on six tokens spread over the
+    batch (the oracle fits each expert in about a minute)."""
+    _moe_case(C.MOE_C5_V2A, tokens=[0, 3, 6, 9, 12, 15])
 
 
 def test_moe_c2_full_all_tokens():
@@ -178,12 +186,12 @@ def test_moe_c4_full_prefill_sampled_tokens():
 
 # The clamp h = silu(min(g, 7)) clamp(u, -7, 7) must act: activations scaled by 16 put
 # at least 10% of the gate values above 7 and 10% of the up values outside [-7, 7].
-_CLAMP = [("mxfp4", 1), ("mxfp4", 2), ("nvfp4", 1), ("nvfp4", 2), ("cb4", 1)]
+_CLAMP = [("mxfp4", 1), ("mxfp4", 2), ("nvfp4", 1), ("nvfp4", 2), ("cb4", 1), ("v2a", 1)]
 
 
 @pytest.mark.parametrize("fmt,variant", _CLAMP, ids=[f"{f}_v{v}" for f, v in _CLAMP])
 def test_moe_clamp_active_small(fmt, variant):
-    base = {"mxfp4": C.MOE_C2, "nvfp4": C.MOE_C3, "cb4": C.MOE_C5}[fmt]
+    base = {"mxfp4": C.MOE_C2, "nvfp4": C.MOE_C3, "cb4": C.MOE_C5, "v2a": C.MOE_C5_V2A}[fmt]
     _moe_case(C.small(base), variant=variant, x_scale=CLAMP_X_SCALE, min_clamp=MIN_CLAMP_SHARE)
 
 
@@ -215,12 +223,13 @@ _EDGE = [
     ("mxfp4", 1, 8, 1, 1), ("mxfp4", 1, 8, 1, 2), ("mxfp4", 5, 4, 4, 1), ("mxfp4", 5, 4, 4, 2),
     ("mxfp4", 3, 1, 1, 2), ("nvfp4", 3, 1, 1, 1), ("nvfp4", 6, 4, 4, 1), ("nvfp4", 1, 8, 1, 2),
     ("nvfp4", 6, 4, 4, 2), ("nvfp4", 3, 1, 1, 2), ("cb4", 2, 1, 1, 1), ("cb4", 4, 4, 4, 1),
+    ("v2a", 2, 1, 1, 1), ("v2a", 4, 4, 4, 1),
 ]
 
 
 @pytest.mark.parametrize("fmt,T,E,k,variant", _EDGE, ids=[f"{f}_t{t}_e{e}_k{k}_v{v}" for f, t, e, k, v in _EDGE])
 def test_moe_edge_routings(fmt, T, E, k, variant):
     from dataclasses import replace
-    base = {"mxfp4": C.MOE_C2, "nvfp4": C.MOE_C3, "cb4": C.MOE_C5}[fmt]
+    base = {"mxfp4": C.MOE_C2, "nvfp4": C.MOE_C3, "cb4": C.MOE_C5, "v2a": C.MOE_C5_V2A}[fmt]
     cfg = replace(base, name=f"edge_{fmt}_t{T}_e{E}_k{k}", T=T, E=E, H=512, I=256, k=k, zipf_bias=False)
     _moe_case(cfg, variant=variant)
