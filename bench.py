@@ -53,7 +53,7 @@ L2_BYTES = 126 * 1024 * 1024
 METRIC = "FP4 MoE layer: decode HBM GB/s (% of peak); prefill TFLOP/s; tokens/s"
 HEADLINE = C.MOE_C4.name
 ORDER = [C.MOE_C4.name, C.LINEAR_C1.name, C.MOE_C2.name, C.MOE_C3.name, C.MOE_C5.name, C.MOE_C4_NV.name,
-         C.MOE_C5_V2A.name]
+         C.MOE_C5_V2A.name, C.MOE_C2_MIXED.name]
 
 
 def parse(argv=None):
@@ -83,7 +83,7 @@ def per_expert_bytes(cfg):
         return (gu + dn) // 2 + (gu + dn) // 4, gu // 2 + gu // 4
     if cfg.fmt == "v2a":       # 4-bit codes + an 8-byte record per 128 weights + a 1 KB library per matrix
         return (gu + dn) // 2 + (gu + dn) // 16 + 2 * 1024, gu // 2 + gu // 16 + 1024
-    B = 32 if cfg.fmt == "mxfp4" else 16
+    B = 32 if cfg.fmt in ("mxfp4", "mixed") else 16       # mixed: the MXFP4 experts (bf16 ones via extra)
     b = (gu + dn) // 2 + (gu + dn) // B
     if cfg.fmt == "nvfp4":
         b += 8
@@ -364,6 +364,8 @@ def run_moe(args, cfg, device, world, peaks):
     w0.kernel_variant = args.variant
     if cfg.fmt in ("mxfp4", "nvfp4") and args.variant != 1:
         prepare_mma_scales(w0)            # one-time weight preparation, outside the timed region
+    elif cfg.fmt == "mixed" and args.variant != 0:
+        w0.kernel_variant = args.variant
     weights = clone_weights(w0, copies)
     structs = [w.c_struct() for w in weights]
     T, k = cfg.T, cfg.k
@@ -388,6 +390,11 @@ def run_moe(args, cfg, device, world, peaks):
     extra_gu = extra_all = None
     if cfg.fmt in ("cb4", "v2a"):
         extra_gu, extra_all = cb4_extra_bytes(w0)
+    if cfg.fmt == "mixed":           # bf16 experts move 2 bytes per weight instead of the MXFP4 bytes
+        gu_d = 2 * (2 * cfg.I * cfg.H) - per_expert_bytes(cfg)[1]
+        all_d = 2 * (3 * cfg.I * cfg.H) - per_expert_bytes(cfg)[0]
+        extra_gu = np.array([gu_d if e in cfg.bf16_experts else 0 for e in range(cfg.E)], dtype=np.int64)
+        extra_all = np.array([all_d if e in cfg.bf16_experts else 0 for e in range(cfg.E)], dtype=np.int64)
     work_step, unit = work_per_step(cfg, counts, extra=extra_all)
     graphs, launches = [], 0
     for c in range(copies):
@@ -473,6 +480,8 @@ def dtype_label(cfg, tensor):
         return "f16(codebook)xf16->f32"
     if cfg.fmt == "v2a":
         return "f16(shared-library codebook)xf16->f32"
+    if cfg.fmt == "mixed":
+        return "f16xe2m1->f32 and bf16xf16->f32 (fp32 FMA)"
     if tensor and cfg.fmt == "mxfp4":
         return "e4m3x2xe2m1->f32"
     return "f16xf16(e2m1*e4m3)->f32" if cfg.fmt == "nvfp4" else "f16xe2m1->f32"
@@ -631,7 +640,8 @@ def _quantise_expert(cfg, which, e):
     """Worker: the oracle's quantised form of one expert matrix (untimed preparation)."""
     from oracle import moe as M
     bank = M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits,
+                            bf16_experts=cfg.bf16_experts)
     return bank.packed(which, e)
 
 
@@ -646,7 +656,8 @@ def oracle_pairs(cfg):
     bias = D.zipf_bias(cfg.seed, cfg.E) if cfg.zipf_bias else None
     ids = R.topk(R.router_logits(x0, wr, bias), cfg.k)[0]
     bank = M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits,
+                            bf16_experts=cfg.bf16_experts)
     jobs = [(which, int(e)) for e in ids for which in ("gu", "dn")]
     with cf.ProcessPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1)),
                                 mp_context=mp.get_context("spawn"), initializer=_limit_threads) as pool:

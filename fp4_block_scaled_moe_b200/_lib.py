@@ -11,7 +11,7 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfp4moe.so")
 
-FP4_MXFP4, FP4_NVFP4, FP4_CB4, FP4_V2A = 1, 2, 3, 4
+FP4_MXFP4, FP4_NVFP4, FP4_CB4, FP4_V2A, FP4_DENSE_BF16 = 1, 2, 3, 4, 5
 FP4_F32, FP4_BF16 = 0, 1
 FORMATS = {"mxfp4": FP4_MXFP4, "nvfp4": FP4_NVFP4, "cb4": FP4_CB4, "v2a": FP4_V2A}
 BLOCK = {FP4_MXFP4: 32, FP4_NVFP4: 16}
@@ -37,6 +37,9 @@ class MoEWeightsC(ctypes.Structure):
         ("kernel_variant", _i32),
         ("gu_mma_scales", _vp), ("dn_mma_scales", _vp),
         ("expert_begin", _i32), ("local_experts", _i32),
+        ("expert_format", _vp), ("gu_offset", _vp), ("gu_scale_offset", _vp), ("dn_offset", _vp),
+        ("dn_scale_offset", _vp), ("gu_bytes", _i64), ("gu_scale_bytes", _i64), ("dn_bytes", _i64),
+        ("dn_scale_bytes", _i64),
     ]
 
 

@@ -234,6 +234,12 @@ class MoEWeights:
     # of the E routed experts (0, 0: all of them)
     expert_begin: int = 0
     local_experts: int = 0
+    # mixed-format fused buffers (see mixed.py): per-expert format and byte offsets
+    expert_format: torch.Tensor | None = None
+    gu_offset: torch.Tensor | None = None
+    gu_scale_offset: torch.Tensor | None = None
+    dn_offset: torch.Tensor | None = None
+    dn_scale_offset: torch.Tensor | None = None
 
     def c_struct(self):
         s = L.MoEWeightsC()
@@ -242,9 +248,13 @@ class MoEWeights:
         s.swiglu_limit = self.swiglu_limit
         s.kernel_variant = self.kernel_variant
         s.expert_begin, s.local_experts = self.expert_begin, self.local_experts
+        if self.expert_format is not None:
+            s.gu_bytes, s.dn_bytes = self.gu_codes.numel(), self.dn_codes.numel()
+            s.gu_scale_bytes, s.dn_scale_bytes = self.gu_scales.numel(), self.dn_scales.numel()
         for name in ("gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales", "dn_tscale", "gu_cb",
                      "gu_rowptr", "gu_col", "gu_val", "dn_cb", "dn_rowptr", "dn_col", "dn_val", "gu_mma_scales",
-                     "dn_mma_scales"):
+                     "dn_mma_scales", "expert_format", "gu_offset", "gu_scale_offset", "dn_offset",
+                     "dn_scale_offset"):
             t = getattr(self, name)
             setattr(s, name, None if t is None else t.data_ptr())
         return s

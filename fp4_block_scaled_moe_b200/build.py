@@ -25,7 +25,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompil
 
 TARGETS = {
     os.path.join(PKG, "libfp4moe.so"): {
-        "srcs": ["api.cu", "pack.cu", "route.cu", "decode.cu", "bs_moe.cu", "nv_moe.cu", "cb4.cu", "v2a.cu", "moe.cu",
+        "srcs": ["api.cu", "pack.cu", "route.cu", "decode.cu", "bs_moe.cu", "nv_moe.cu", "cb4.cu", "v2a.cu", "dense16.cu", "moe.cu",
                  "no_alloc.cu"],
         "dir": os.path.join(PKG, "csrc"),
         "inc": [os.path.join(ROOT, "include"), os.path.join(PKG, "csrc")],

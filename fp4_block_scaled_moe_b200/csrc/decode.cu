@@ -81,11 +81,16 @@ struct Unit {
 
 // Exclusive scans by warp 0 over E experts: off = scan(cnt), pre = scan(units per expert),
 // where only the experts in [e_lo, e_hi) (those whose weights the call holds) have units.
-__device__ void scan_experts(const int* cnt, int* off, int* pre, int E, int tiles, int e_lo, int e_hi) {
+// In a mixed-format buffer (ex_fmt non-null) only the experts of format `want` have units.
+__device__ void scan_experts(const int* cnt, int* off, int* pre, int E, int tiles, int e_lo, int e_hi,
+                             const uint8_t* ex_fmt, int want) {
   const int lane = threadIdx.x & 31;
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-  auto units = [&](int e) { return (e >= e_lo && e < e_hi) ? (cnt[e] + kTok - 1) / kTok * tiles : 0; };
+  auto units = [&](int e) {
+    const bool mine = e >= e_lo && e < e_hi && (ex_fmt == nullptr || ex_fmt[e - e_lo] == want);
+    return mine ? (cnt[e] + kTok - 1) / kTok * tiles : 0;
+  };
   int sc = 0, su = 0;
   for (int e = e0; e < e1; ++e) {
     sc += cnt[e];
@@ -139,12 +144,31 @@ __device__ __forceinline__ Unit unit_static(int u, int tiles, int T) {
   return un;
 }
 
+// row of the expert's matrix that row r (0..63) of a unit reads
+template <int kEpi>
+__device__ __forceinline__ int64_t tile_row(const DecodeArgs& a, const Unit& un, int r) {
+  if (kEpi == kEpiSwiglu) return r < 32 ? un.tile * 32 + r : a.inter + un.tile * 32 + (r - 32);
+  return static_cast<int64_t>(un.tile) * kRows + r;
+}
+// first code row and first scale row of the unit's expert (rows of K/2 code bytes and of
+// the per-row scale bytes): uniform buffers stack the local experts; mixed-format buffers
+// give each expert's byte offsets
+struct RowBase {
+  int64_t code, scale;
+};
+template <int kFmt>
+__device__ __forceinline__ RowBase unit_base(const DecodeArgs& a, const Unit& un) {
+  const int le = un.e - a.e_begin;
+  if (a.row_off == nullptr) {
+    const int64_t b = static_cast<int64_t>(le) * a.rows_per_expert;
+    return {b, b};
+  }
+  constexpr int kB = (kFmt == FP4_MXFP4) ? 32 : 16;
+  return {a.row_off[le] / (a.K / 2), a.srow_off[le] / (a.K / kB)};
+}
 template <int kEpi>
 __device__ __forceinline__ int64_t unit_row(const DecodeArgs& a, const Unit& un, int r) {
-  const int64_t base = static_cast<int64_t>(un.e - a.e_begin) * a.rows_per_expert;   // local expert
-  if (kEpi == kEpiSwiglu)
-    return base + (r < 32 ? un.tile * 32 + r : a.inter + un.tile * 32 + (r - 32));
-  return base + static_cast<int64_t>(un.tile) * kRows + r;
+  return static_cast<int64_t>(un.e - a.e_begin) * a.rows_per_expert + tile_row<kEpi>(a, un, r);   // local expert
 }
 
 // CB4: eight 4-bit indices (low nibble first) -> four f16x2 registers of codebook
@@ -179,7 +203,8 @@ __device__ __forceinline__ void cb4_lookup8(uint32_t w, const uint32_t (&lo)[4],
 
 template <int kFmt, int kEpi, int kMode, int KC>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
-    decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a, const Layout L) {
+    decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap smap,
+                  const DecodeArgs a, const Layout L) {
   // stage geometry (must match make_layout)
   constexpr bool kCb = (kFmt == FP4_CB4 || kFmt == FP4_V2A);      // codebook lookup formats
   constexpr int kB = (kFmt == FP4_MXFP4) ? 32 : 16;
@@ -216,7 +241,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   if (kFmt == FP4_MXFP4)
     for (int i = threadIdx.x; i < 256; i += kThreads)
       reinterpret_cast<float*>(smem + L.lut_off)[i] = ue8m0_to_f32(static_cast<uint32_t>(i));
-  if (warp == kConsumers && lane == 0) prefetch_tmap(&tmap);
+  if (warp == kConsumers && lane == 0) {
+    prefetch_tmap(&tmap);
+    if (a.scale_tma) prefetch_tmap(&smap);
+  }
   __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
@@ -245,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
       }
       __syncthreads();
       if (warp == 0) {
-        scan_experts(cnt, off, pre, E, tiles, a.e_begin, a.e_end);
+        scan_experts(cnt, off, pre, E, tiles, a.e_begin, a.e_end, a.ex_fmt, kFmt);
         __syncwarp();
         // stable placement: pairs in ascending order, 32 per round, ranked within the round
         int* cur = pre + E + 1;                      // [E] cursors
@@ -280,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     } else {
       for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = a.counts[e];
       __syncthreads();
-      if (warp == 0) scan_experts(cnt, off, pre, E, tiles, a.e_begin, a.e_end);
+      if (warp == 0) scan_experts(cnt, off, pre, E, tiles, a.e_begin, a.e_end, a.ex_fmt, kFmt);
       __syncthreads();
     }
     n_units = pre[E];
@@ -323,10 +351,14 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         break;
       }
       const Unit un = get_unit(u);
-      const int64_t y0 = unit_row<kEpi>(a, un, 0), y1 = unit_row<kEpi>(a, un, 32);
+      const RowBase rb0 = unit_base<kFmt>(a, un);
+      const int64_t y0 = rb0.code + tile_row<kEpi>(a, un, 0), y1 = rb0.code + tile_row<kEpi>(a, un, 32);
+      const int64_t sy0 = rb0.scale + tile_row<kEpi>(a, un, 0), sy1 = rb0.scale + tile_row<kEpi>(a, un, 32);
       int xr = 0;
       if (lane < un.ntok) xr = (kEpi == kEpiSwiglu) ? perm_at(un.slot0 + lane) / a.topk : un.slot0 + lane;
-      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2 + (kCb ? kRows * kScaleRow : 0) +
+      const bool stma = a.scale_tma != 0;   // the per-row scale bytes arrive as two TMA boxes
+      const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2 +
+                                                ((kCb || stma) ? kRows * kScaleRow : 0) +
                                                 (kFmt == FP4_V2A ? kV2aLibBytes : 0));
       constexpr int words = kScaleRow / 4;
       for (int c = 0; c < L.nchunks; ++c, ++it) {
@@ -339,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st_base = sbase + s * L.stage_bytes;
         const int k0 = c * KC;
-        if (!kCb) {
+        if (!kCb && !stma) {
           for (int w = lane; w < kRows * words; w += 32) {
             const int r = w / words, cw = w - r * words;
-            const uint8_t* src = a.scales + unit_row<kEpi>(a, un, r) * (a.K / B) + k0 / B + cw * 4;
+            const uint8_t* src = a.scales + (rb0.scale + tile_row<kEpi>(a, un, r)) * (a.K / B) + k0 / B + cw * 4;
             cp_async4(st_base + kScalesOff + r * kScaleRow + cw * 4, src);
           }
           cp_async_arrive(bar_full + 8 * s);
@@ -350,10 +382,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         __syncwarp();
-        if (kCb)
+        if (stma) {
+          // rows 0-31 and 32-63 of the unit (gate_up: the gate and the up block) as two boxes
+          if (lane == 0) {
+            const int32_t sx = k0 / (KC / kScaleRow);
+            tma_load_2d(st_base + kScalesOff, &smap, sx, static_cast<int32_t>(sy0), bar_full + 8 * s);
+            tma_load_2d(st_base + kScalesOff + 32 * kScaleRow, &smap, sx, static_cast<int32_t>(sy1), bar_full + 8 * s);
+          }
+        } else if (kCb)
           for (int r = lane; r < kRows; r += 32)
             bulk_g2s(st_base + kScalesOff + r * kScaleRow,
-                     a.scales + unit_row<kEpi>(a, un, r) * (a.K / (KC / kScaleRow)) + k0 / (KC / kScaleRow),
+                     a.scales + (rb0.scale + tile_row<kEpi>(a, un, r)) * (a.K / (KC / kScaleRow)) + k0 / (KC / kScaleRow),
                      static_cast<uint32_t>(kScaleRow), bar_full + 8 * s);
         if (kFmt == FP4_V2A && lane == 0)
           bulk_g2s(st_base + kLibOff, a.lib + static_cast<int64_t>(un.e - a.e_begin) * kV2aLibBytes, kV2aLibBytes,
@@ -632,34 +671,34 @@ Layout make_layout(int fmt, int K, int E, int P, int P_scl) {
 }
 
 template <int kFmt, int kEpi, int kMode, int KC>
-fp4_status launch_kc(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
-                     bool pdl) {
+fp4_status launch_kc(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, const CUtensorMap& smap, int grid,
+                     cudaStream_t st, bool pdl) {
   auto kern = decode_kernel<kFmt, kEpi, kMode, KC>;
   static thread_local int configured = 0;
   if (configured < L.smem_bytes) {
     FP4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem_bytes));
     configured = L.smem_bytes;
   }
-  return launch_pdl(kern, dim3(grid), dim3(kThreads), static_cast<size_t>(L.smem_bytes), st, pdl, map, a, L);
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), static_cast<size_t>(L.smem_bytes), st, pdl, map, smap, a, L);
 }
 
 template <int kFmt, int kEpi, int kMode>
-fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
-                      bool pdl) {
+fp4_status launch_one(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, const CUtensorMap& smap,
+                      int grid, cudaStream_t st, bool pdl) {
   if constexpr (kFmt != FP4_CB4 && kFmt != FP4_V2A) {
-    if (L.kc == 512) return launch_kc<kFmt, kEpi, kMode, 512>(a, L, map, grid, st, pdl);
+    if (L.kc == 512) return launch_kc<kFmt, kEpi, kMode, 512>(a, L, map, smap, grid, st, pdl);
   }
-  return launch_kc<kFmt, kEpi, kMode, 256>(a, L, map, grid, st, pdl);
+  return launch_kc<kFmt, kEpi, kMode, 256>(a, L, map, smap, grid, st, pdl);
 }
 
 template <int kFmt>
-fp4_status dispatch(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, int grid, cudaStream_t st,
-                    bool pdl) {
+fp4_status dispatch(const DecodeArgs& a, const Layout& L, const CUtensorMap& map, const CUtensorMap& smap, int grid,
+                    cudaStream_t st, bool pdl) {
   if (a.epi == kEpiSwiglu && a.mode == kModeRoute)
-    return launch_one<kFmt, kEpiSwiglu, kModeRoute>(a, L, map, grid, st, pdl);
-  if (a.epi == kEpiSwiglu) return launch_one<kFmt, kEpiSwiglu, kModeList>(a, L, map, grid, st, pdl);
-  if (a.epi == kEpiDown) return launch_one<kFmt, kEpiDown, kModeList>(a, L, map, grid, st, pdl);
-  return launch_one<kFmt, kEpiLinear, kModeStatic>(a, L, map, grid, st, pdl);
+    return launch_one<kFmt, kEpiSwiglu, kModeRoute>(a, L, map, smap, grid, st, pdl);
+  if (a.epi == kEpiSwiglu) return launch_one<kFmt, kEpiSwiglu, kModeList>(a, L, map, smap, grid, st, pdl);
+  if (a.epi == kEpiDown) return launch_one<kFmt, kEpiDown, kModeList>(a, L, map, smap, grid, st, pdl);
+  return launch_one<kFmt, kEpiLinear, kModeStatic>(a, L, map, smap, grid, st, pdl);
 }
 
 }  // namespace
@@ -675,10 +714,22 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
                           static_cast<uint64_t>(a.K / 2), 128, 32, CU_TENSOR_MAP_SWIZZLE_128B));
   int grid = ctas_per_sm(L.kc) * num_sms();
   if (a.mode == kModeStatic) grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok));
-  if (a.fmt == FP4_CB4) return dispatch<FP4_CB4>(a, L, map, grid, st, pdl);
-  if (a.fmt == FP4_V2A) return dispatch<FP4_V2A>(a, L, map, grid, st, pdl);
-  return (a.fmt == FP4_NVFP4) ? dispatch<FP4_NVFP4>(a, L, map, grid, st, pdl)
-                              : dispatch<FP4_MXFP4>(a, L, map, grid, st, pdl);
+  // the per-row scale bytes (E2M1 block scales, CB4 codebooks, V2a group records) by TMA
+  // when a stage's share of a row and the row stride are multiples of 16 bytes
+  DecodeArgs b = a;
+  const int64_t k_per_byte = L.kc / L.scale_row;                     // K elements per scale byte
+  const int64_t srow = a.K / k_per_byte;                             // scale bytes per row
+  b.scale_tma = (L.scale_row % 16 == 0 && srow % 16 == 0) ? 1 : 0;
+  CUtensorMap smap = map;
+  if (b.scale_tma)
+    FP4_TRY(make_tmap_2d_u8(&smap, a.scales, static_cast<uint64_t>(srow),
+                            static_cast<uint64_t>(a.scale_rows_total > 0 ? a.scale_rows_total : a.rows_total),
+                            static_cast<uint64_t>(srow), static_cast<uint32_t>(L.scale_row), 32,
+                            CU_TENSOR_MAP_SWIZZLE_NONE));
+  if (a.fmt == FP4_CB4) return dispatch<FP4_CB4>(b, L, map, smap, grid, st, pdl);
+  if (a.fmt == FP4_V2A) return dispatch<FP4_V2A>(b, L, map, smap, grid, st, pdl);
+  return (a.fmt == FP4_NVFP4) ? dispatch<FP4_NVFP4>(b, L, map, smap, grid, st, pdl)
+                              : dispatch<FP4_MXFP4>(b, L, map, smap, grid, st, pdl);
 }
 
 // y[t, n] = bf16( sum_{j = 0..k-1} o[inv[t k + j], n] ), fixed j order (deterministic).

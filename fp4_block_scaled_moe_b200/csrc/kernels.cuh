@@ -93,6 +93,13 @@ struct DecodeArgs {
   int32_t* perm;                 // [P] slot -> pair
   int32_t* inv;                  // [P] pair -> slot (written by CTA 0 in kModeRoute)
   int static_tiles;              // linear: N / 64
+  int scale_tma;                 // set by launch_decode: scale bytes by TMA boxes (else per-row copies)
+  // mixed-format fused buffers (or null): per local expert its format and the byte offsets of
+  // its rows in `codes` and `scales`; only experts of this kernel's format get units
+  const uint8_t* ex_fmt;
+  const int64_t* row_off;
+  const int64_t* srow_off;
+  int64_t scale_rows_total;      // mixed-format buffers: rows of the scale buffer (else rows_total)
   const __half* x16;             // activation rows, f16 [rows, K]
   const int* sexp;               // per token exponent (swiglu / linear) or null
   float limit;                   // swiglu clamp
@@ -106,6 +113,26 @@ struct DecodeArgs {
 };
 
 fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl);
+
+// The bf16 experts of a mixed-format fused buffer (dense16.cu): same units and epilogues
+// as the grouped GEMV; weights at weights + offset[e - e_begin], bf16 rows of K.
+struct Dense16Args {
+  int epi;
+  const uint8_t* weights;
+  const int64_t* offset;
+  const uint8_t* ex_fmt;
+  int e_begin, e_end, E, K, rows_per_expert, inter, topk;
+  const int32_t* counts;
+  const int32_t* perm;
+  const __half* x16;          // gate_up: token rows (scaled by 2^sexp); down: h rows by slot
+  const int* sexp;
+  float limit;
+  __half* h_out;
+  const float* gw;
+  float* o_out;
+  int ldo;
+};
+fp4_status launch_dense16(const Dense16Args& a, cudaStream_t st);
 
 // y[t, :] = bf16(sum_j o[inv[t k + j], :]) in j order.
 __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv, int T, int k, int H,

@@ -29,6 +29,7 @@ bool tensor_supported(const fp4_moe_weights* w, int32_t T) {
 }
 
 int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
+  if (w->expert_format != nullptr) return kVarGemv;      // mixed-format buffers: CUDA-core kernels
   const bool tc_ok = tensor_supported(w, T);
   if (w->kernel_variant == kVarTensor) return kVarTensor;
   if (w->kernel_variant == kVarGemv) return kVarGemv;
@@ -150,6 +151,15 @@ fp4_status check_moe(const fp4_moe_weights* w, int32_t T, int32_t k) {
   }
   if (!w->gu_codes || !w->gu_scales || !w->dn_codes || !w->dn_scales) return FP4_ERR_INVALID_ARG;
   if (w->fmt == FP4_NVFP4 && (!w->gu_tscale || !w->dn_tscale)) return FP4_ERR_INVALID_ARG;
+  if (w->expert_format != nullptr) {
+    if (w->fmt != FP4_MXFP4) return FP4_ERR_UNSUPPORTED;
+    if (!w->gu_offset || !w->gu_scale_offset || !w->dn_offset || !w->dn_scale_offset) return FP4_ERR_INVALID_ARG;
+    if (w->gu_bytes <= 0 || w->dn_bytes <= 0 || w->gu_scale_bytes <= 0 || w->dn_scale_bytes <= 0)
+      return FP4_ERR_EMPTY_SHAPE;
+    if (w->gu_bytes % (H / 2) || w->dn_bytes % (I / 2) || w->gu_scale_bytes % (H / 32) || w->dn_scale_bytes % (I / 32))
+      return FP4_ERR_ALIGNMENT;
+    if (w->kernel_variant == kVarTensor) return FP4_ERR_UNSUPPORTED;
+  }
   if (w->kernel_variant < 0 || w->kernel_variant > 2) return FP4_ERR_INVALID_ARG;
   if (w->kernel_variant == kVarTensor && !tensor_supported(w, T)) return FP4_ERR_UNSUPPORTED;
   if (!aligned16(w->gu_codes) || !aligned16(w->gu_scales) || !aligned16(w->dn_codes) || !aligned16(w->dn_scales))
@@ -375,13 +385,18 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
     g.sp_col = w->gu_col;
     g.sp_val = w->gu_val;
   }
-  g.rows_total = static_cast<int64_t>(El) * 2 * I;
+  const bool mixed = w->expert_format != nullptr;
+  g.rows_total = mixed ? w->gu_bytes / (H / 2) : static_cast<int64_t>(El) * 2 * I;
   g.K = H;
   g.rows_per_expert = 2 * I;
   g.inter = I;
   g.E = E;
   g.e_begin = e0;
   g.e_end = e1;
+  g.ex_fmt = w->expert_format;
+  g.row_off = w->gu_offset;
+  g.srow_off = w->gu_scale_offset;
+  g.scale_rows_total = mixed ? w->gu_scale_bytes / (H / 32) : 0;
   g.T = T;
   g.topk = k;
   g.logits = ra.logits;
@@ -400,6 +415,27 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
   g.slot = &ra.ctrl->slot[0];
   g.unit_next = &ra.ctrl->unit_next[0];
   FP4_TRY(launch_decode(g, st, true));
+  Dense16Args dg{};
+  if (mixed) {                     // the bf16 experts of the mixed buffer, same units and epilogue
+    dg.epi = kEpiSwiglu;
+    dg.weights = w->gu_codes;
+    dg.offset = w->gu_offset;
+    dg.ex_fmt = w->expert_format;
+    dg.e_begin = e0;
+    dg.e_end = e1;
+    dg.E = E;
+    dg.K = H;
+    dg.rows_per_expert = 2 * I;
+    dg.inter = I;
+    dg.topk = k;
+    dg.counts = ra.counts;
+    dg.perm = ra.perm;
+    dg.x16 = ra.x16;
+    dg.sexp = ra.sexp;
+    dg.limit = w->swiglu_limit;
+    dg.h_out = g.h_out;
+    FP4_TRY(launch_dense16(dg, st));
+  }
 
   DecodeArgs d = g;
   d.epi = kEpiDown;
@@ -413,9 +449,12 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
     d.sp_col = w->dn_col;
     d.sp_val = w->dn_val;
   }
-  d.rows_total = static_cast<int64_t>(El) * H;
+  d.rows_total = mixed ? w->dn_bytes / (I / 2) : static_cast<int64_t>(El) * H;
   d.K = I;
   d.rows_per_expert = H;
+  d.row_off = w->dn_offset;
+  d.srow_off = w->dn_scale_offset;
+  d.scale_rows_total = mixed ? w->dn_scale_bytes / (I / 32) : 0;
   d.x16 = g.h_out;
   d.sexp = nullptr;
   d.o_out = reinterpret_cast<float*>(ws + L.o);
@@ -423,6 +462,21 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
   d.unit_next = &ra.ctrl->unit_next[1];
   d.ldo = H;
   FP4_TRY(launch_decode(d, st, true));
+  if (mixed) {
+    Dense16Args dd = dg;
+    dd.epi = kEpiDown;
+    dd.weights = w->dn_codes;
+    dd.offset = w->dn_offset;
+    dd.K = I;
+    dd.rows_per_expert = H;
+    dd.x16 = g.h_out;
+    dd.sexp = nullptr;
+    dd.h_out = nullptr;
+    dd.gw = ra.gw;
+    dd.o_out = d.o_out;
+    dd.ldo = H;
+    FP4_TRY(launch_dense16(dd, st));
+  }
   return launch_combine(d.o_out, ra.inv, ra.ids, T, k, H, e0, e1, y_bf16, y_partial, st);
 }
 

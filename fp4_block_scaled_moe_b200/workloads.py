@@ -48,8 +48,23 @@ def device_weights_v2a(cfg, device="cuda"):
                       dn_cb=dn["lib"], dn_rowptr=dn["row_ptr"], dn_col=dn["col"], dn_val=dn["val"])
 
 
+def device_weights_mixed(cfg, device="cuda"):
+    """A mixed-format fused buffer: the experts in cfg.bf16_experts kept in bf16, the rest
+    MXFP4 (see mixed.py)."""
+    from .mixed import pack_mixed
+    ws = {}
+    for which, tid, rows, K in (("gu", C.TID_GATE_UP, 2 * cfg.I, cfg.H), ("dn", C.TID_DOWN, cfg.H, cfg.I)):
+        w = torch.empty((cfg.E, rows, K), dtype=torch.float32, device=device)
+        SD.expert_weights_into(w.view(cfg.E * rows, K), cfg.seed, tid, start_row=0, sigma=cfg.sigma,
+                               outliers=cfg.outliers)
+        ws[which] = w
+    return pack_mixed(ws["gu"], ws["dn"], cfg.bf16_experts, cfg.swiglu_limit)
+
+
 def device_weights(cfg, device="cuda", chunk_elems=1 << 28):
     """Draw every expert's weights of ``cfg`` on the device and pack them there."""
+    if cfg.fmt == "mixed":
+        return device_weights_mixed(cfg, device)
     if cfg.fmt == "cb4":
         return device_weights_cb4(cfg, device)
     if cfg.fmt == "v2a":

@@ -66,7 +66,13 @@ typedef enum fp4_status {
   FP4_ERR_TIMEOUT = 8         /* a bounded device-side wait gave up */
 } fp4_status;
 
-typedef enum fp4_format { FP4_MXFP4 = 1, FP4_NVFP4 = 2, FP4_CB4 = 3, FP4_V2A = 4 } fp4_format;
+typedef enum fp4_format {
+  FP4_MXFP4 = 1,
+  FP4_NVFP4 = 2,
+  FP4_CB4 = 3,
+  FP4_V2A = 4,
+  FP4_DENSE_BF16 = 5 /* an expert kept in bf16 inside a mixed-format buffer (expert_format) */
+} fp4_format;
 
 typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
 
@@ -245,6 +251,27 @@ typedef struct fp4_moe_weights {
    * outside [0, E] is FP4_ERR_INVALID_ARG. */
   int32_t expert_begin;
   int32_t local_experts;
+  /* Mixed formats in one fused buffer ("The gate that missed by 0.0202 pp", section "A fused
+   * tensor with two dtypes in it": a fused MoE buffer packs every expert of a layer into one
+   * tensor, an expert excluded from quantisation keeps its full-width bf16 rows beside the
+   * half-width packed experts, so the format and the stride belong to the expert, not to the
+   * tensor).  When expert_format is non-NULL (device uint8 [local experts]), fmt must be
+   * FP4_MXFP4 and each expert is FP4_MXFP4 or FP4_DENSE_BF16:
+   *   *_codes    one fused byte buffer of *_bytes bytes; expert e's rows start at byte
+   *              *_offset[e] (device int64 [local experts], a multiple of K/2 with K = H for
+   *              gate_up, I for down): MXFP4 codes [rows, K/2] or bf16 [rows, K];
+   *   *_scales   one fused buffer of *_scale_bytes bytes holding the MXFP4 experts' scales
+   *              [rows, K/32] at *_scale_offset[e] (a multiple of K/32; unused for bf16).
+   * Such layers run on the CUDA-core kernels (kernel_variant 2 is FP4_ERR_UNSUPPORTED). */
+  const uint8_t* expert_format;
+  const int64_t* gu_offset;
+  const int64_t* gu_scale_offset;
+  const int64_t* dn_offset;
+  const int64_t* dn_scale_offset;
+  int64_t gu_bytes;
+  int64_t gu_scale_bytes;
+  int64_t dn_bytes;
+  int64_t dn_scale_bytes;
 } fp4_moe_weights;
 
 /*

@@ -80,25 +80,29 @@ class LazyExpertBank:
     "dn" -> [H, I]); they are quantised here with this package's own formats (MXFP4,
     NVFP4 with one tensor scale per expert matrix, CB4 or V2a (``v2a_bits`` per code,
     one library per expert matrix) with ``cb4_threshold`` as the absolute outlier
-    threshold around mu = 0) and dequantised exactly in float64.
+    threshold around mu = 0, or "mixed": MXFP4 except the ``bf16_experts``, which are
+    rounded to bf16) and dequantised exactly in float64.
     """
 
-    def __init__(self, fmt, E, H, I, draw, cb4_threshold=None, v2a_bits=4):
+    def __init__(self, fmt, E, H, I, draw, cb4_threshold=None, v2a_bits=4, bf16_experts=()):
         self.fmt, self.E, self.H, self.I = fmt, E, H, I
         self.draw = draw
         self.cb4_threshold = cb4_threshold
         self.v2a_bits = v2a_bits
+        self.bf16_experts = set(bf16_experts)
         self._cache = {}
 
     def packed(self, which, e):
         key = (which, e)
         if key not in self._cache:
             w = self.draw(which, e)
-            if self.fmt == "cb4":
+            if self.fmt == "mixed" and e in self.bf16_experts:
+                self._cache[key] = ("bf16", formats.round_to_bf16(w.astype(np.float64)))
+            elif self.fmt == "cb4":
                 self._cache[key] = codebook.cb4_fit(w, self.cb4_threshold)
             elif self.fmt == "v2a":
                 self._cache[key] = v2a.v2a_fit(w, self.v2a_bits, self.cb4_threshold)
-            elif self.fmt == "mxfp4":
+            elif self.fmt in ("mxfp4", "mixed"):
                 self._cache[key] = formats.mxfp4_quantize(w) + (None,)
             else:
                 c, s, t = formats.nvfp4_quantize(w[None])
@@ -106,6 +110,8 @@ class LazyExpertBank:
         return self._cache[key]
 
     def dequant(self, which, e):
+        if self.fmt == "mixed" and e in self.bf16_experts:
+            return self.packed(which, e)[1]
         if self.fmt == "v2a":
             return v2a.v2a_matrix(self.packed(which, e), self.H if which == "gu" else self.I)
         if self.fmt == "cb4":
@@ -114,7 +120,7 @@ class LazyExpertBank:
             return (codebook.cb4_dense(fit["idx"], fit["cb_val"])
                     + codebook.cb4_sparse(fit["row_ptr"], fit["col"], fit["val"], n, 2 * k2))
         c, s, t = self.packed(which, e)
-        if self.fmt == "mxfp4":
+        if self.fmt in ("mxfp4", "mixed"):
             return formats.mxfp4_dequantize(c, s)
         return formats.nvfp4_dequantize(c, s, t)
 

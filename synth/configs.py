@@ -48,6 +48,8 @@ class MoEConfig:
     cb4_threshold_sigma: float = 6.0
     # V2a: bits per code (N)
     v2a_bits: int = 4
+    # mixed-format buffers: experts kept in bf16 (the rest MXFP4)
+    bf16_experts: tuple = ()
     swiglu_limit: float = 7.0
     seed: int = SEED
     sigma: float = SIGMA
@@ -76,7 +78,12 @@ MOE_C4_NV = MoEConfig("moe_nvfp4_prefill_e256_h6144_i2048_k8_t8192", "nvfp4", T=
 MOE_C5_V2A = MoEConfig("moe_v2a4_decode_e64_h2048_i768_k8_t16", "v2a", T=16, E=64, H=2048, I=768, k=8,
                        outliers=(0.00394, 6.0, 49.0))
 
-FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5, MOE_C4_NV, MOE_C5_V2A)}
+# A mixed-format fused buffer: the MXFP4 decode layer with five experts excluded from
+# quantisation and kept in bf16 (full-width rows) inside the same fused tensor.
+MOE_C2_MIXED = MoEConfig("moe_mixed_mxfp4_bf16_decode_e64_h2048_i768_k8_t16", "mixed", T=16, E=64, H=2048, I=768,
+                         k=8, bf16_experts=(3, 6, 11, 42, 60))
+
+FULL = {c.name: c for c in (LINEAR_C1, MOE_C2, MOE_C3, MOE_C4, MOE_C5, MOE_C4_NV, MOE_C5_V2A, MOE_C2_MIXED)}
 # The prefill layer at a quarter of the experts and tokens (same per-expert load, same
 # tile shapes; 1.3 GB of weights): the size used for full hardware-counter captures.
 MOE_C4_PROFILE = MoEConfig("moe_mxfp4_prefill_e64_h6144_i2048_k8_t2048", "mxfp4", T=2048, E=64, H=6144,
@@ -96,6 +103,9 @@ def small(cfg):
         return replace(cfg, name=cfg.name + "_small", T=5, N=320, K=768)
     if cfg.fmt in ("cb4", "v2a"):
         return replace(cfg, name=cfg.name + "_small", T=7, E=8, H=512, I=256, k=3)
+    if cfg.fmt == "mixed":
+        return replace(cfg, name=cfg.name + "_small", T=9, E=16, H=768, I=512, k=4,
+                       bf16_experts=tuple(e for e in cfg.bf16_experts if e < 16))
     if cfg.T > 1000:  # prefill-shaped: many tokens per expert
         return replace(cfg, name=cfg.name + "_small", T=300, E=8, H=512, I=256, k=2)
     return replace(cfg, name=cfg.name + "_small", T=9, E=16, H=768, I=512, k=4)

@@ -76,7 +76,8 @@ def oracle_bank(cfg):
     """The oracle's lazily quantised expert bank for a workload (host draws)."""
     from oracle import moe as M
     return M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits,
+                            bf16_experts=cfg.bf16_experts)
 
 
 LazyOracleBank = oracle_bank

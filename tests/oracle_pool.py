@@ -43,7 +43,8 @@ def _expert_task(cfg, e, x_rows, limit, corrupt=None):
     from oracle import moe as M
     from synth import configs as C
     bank = M.LazyExpertBank(cfg.fmt, cfg.E, cfg.H, cfg.I, draw=functools.partial(C.expert_rows, cfg),
-                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits)
+                            cb4_threshold=cfg.cb4_threshold_sigma * cfg.sigma, v2a_bits=cfg.v2a_bits,
+                            bf16_experts=cfg.bf16_experts)
     if corrupt is not None:
         corrupt(bank, e)
     gu = bank.apply_gate_up(int(e), x_rows)

@@ -103,6 +103,16 @@ def test_moe_small(cfg):
     _moe_case(cfg)
 
 
+@pytest.mark.parametrize("cfg", [C.small(C.MOE_C2_MIXED), C.MOE_C2_MIXED], ids=["small", "full"])
+def test_moe_mixed_format_buffer(cfg):
+    """A fused buffer holding MXFP4 experts and bf16 experts (kept out of quantisation),
+    each at its own offset: every token, and both kinds of expert are routed."""
+    routed = set(np.unique(R.topk(R.router_logits(D.bf16_bits_to_f32(host_small_inputs(cfg)[0]),
+                                                  host_small_inputs(cfg)[1]), cfg.k)).tolist())
+    assert routed & set(cfg.bf16_experts) and routed - set(cfg.bf16_experts)
+    _moe_case(cfg)
+
+
 def test_moe_v2a_full_sampled_tokens():
     """The V2a layer at full size (the CB4 layer's dimensions and outliers, 4-bit codes
     into one shared 32-codebook library per expert matrix), on six tokens spread over the
