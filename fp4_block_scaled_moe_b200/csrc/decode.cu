@@ -430,6 +430,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   uint32_t c_xo[kNq];
 #pragma unroll
   for (int jj = 0; jj < kNq; ++jj) c_xo[jj] = static_cast<uint32_t>((((jbase & 7) + jj) ^ g) << 4);
+  // NVFP4: byte-permute selectors taking scale byte b of two rows' words into bytes 0, 1
+  // (b = t / 2 for even regions, 2 + t / 2 for odd ones)
+  const uint32_t nv_sel[2] = {static_cast<uint32_t>((t >> 1) | ((4 + (t >> 1)) << 4)),
+                              static_cast<uint32_t>((2 + (t >> 1)) | ((6 + (t >> 1)) << 4))};
   const uint32_t s_off = kScalesOff + rbase * kScaleRow +
                          (kFmt == FP4_MXFP4 ? jbase
                                             : (kFmt == FP4_NVFP4 ? 2 * jbase : (jbase >> 2) * (kFmt == FP4_CB4 ? 32 : 8)));
@@ -533,16 +537,12 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
             mma_16816(acc[mt], p[2 * mt][2], p[2 * mt + 1][2], p[2 * mt][3], p[2 * mt + 1][3], xq.z, xq.w);
           }
         } else if (kFmt == FP4_NVFP4) {
-          // this thread's 8 K positions lie in block 2j + (t >> 1): byte 2 jj + (t >> 1) of the row's run
-          const int bsel = 2 * jj + (t >> 1);
-          uint32_t b4[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t word = (bsel < 4) ? sb[m][0] : sb[m][(kFmt == FP4_MXFP4) ? 0 : 1];
-            b4[m] = (word >> (8 * (bsel & 3))) & 0xFFu;
-          }
-          const uint32_t s01 = e4m3x2_to_f16x2(b4[0] | (b4[1] << 8));
-          const uint32_t s23 = e4m3x2_to_f16x2(b4[2] | (b4[3] << 8));
+          // this thread's 8 K positions lie in block 2 jj + (t >> 1): byte (2 jj + (t >> 1)) & 3 of
+          // word jj / 2 of the row's run; one byte-permute gathers it for two rows at once
+          const int wi = (kFmt == FP4_NVFP4) ? (jj >> 1) : 0;
+          const uint32_t sel = nv_sel[jj & 1];
+          const uint32_t s01 = e4m3x2_to_f16x2(__byte_perm(sb[0][wi], sb[1][wi], sel));
+          const uint32_t s23 = e4m3x2_to_f16x2(__byte_perm(sb[2][wi], sb[3][wi], sel));
           const uint32_t sc[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
                                   __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
 #pragma unroll
