@@ -229,10 +229,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   int* pre = reinterpret_cast<int*>(smem + L.pre_off);
   int* perm_s = reinterpret_cast<int*>(smem + L.perm_off);
 
+  // dense layer with bf16 x: the producer converts x itself (no separate launch) and streams
+  // the weights before waiting on the previous kernel (they do not depend on it)
+  const bool fused_x = kMode == kModeStatic && a.x16 == nullptr;
   __shared__ unsigned int exit_count;
   if (threadIdx.x == 0) {
     for (int s = 0; s < L.stages; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, fused_x ? 2 : 1);   // fused: the weight bytes, then the x rows
       mbar_init(bar_empty + 8 * s, kConsumers);
     }
     fence_barrier_init();
@@ -246,9 +249,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     if (a.scale_tma) prefetch_tmap(&smap);
   }
   __syncthreads();
-  pdl_wait();
+  if (!fused_x) pdl_wait();
   pdl_launch_dependents();
-  if (threadIdx.x == 0) slot_begin(a.slot);
+  // (fused dense layer: the producer starts the timer after its dependency wait, when the
+  // previous launch -- which may share the workspace -- has finished)
+  if (threadIdx.x == 0 && !fused_x) slot_begin(a.slot);
   auto finish = [&]() {   // the last warp of the CTA to leave records the CTA's end time
     if (lane == 0 && atomicAdd(&exit_count, 1u) == kConsumers) slot_end(a.slot);
   };
@@ -330,6 +335,142 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     if (lane == 0) v = static_cast<int>(gridDim.x + atomicAdd(a.unit_next, 1u));
     return __shfl_sync(0xFFFFFFFFu, v, 0);
   };
+
+  if (kMode == kModeStatic && warp == kConsumers && fused_x) {
+    // ------------------------- producer, dense layer with bf16 x ----------------------
+    float* scl_w = reinterpret_cast<float*>(smem + L.scl_off);
+    const bool stma = a.scale_tma != 0;
+    constexpr int words = kScaleRow / 4;
+    const uint32_t wtx = static_cast<uint32_t>(kRows * (KC / 2) + (stma ? kRows * kScaleRow : 0));
+    const int S = L.stages;
+    int it = 0;
+    bool ok = true, waited = false;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit un = get_unit(u);
+      const RowBase rb0 = unit_base<kFmt>(a, un);
+      const int64_t y0 = rb0.code + tile_row<kEpi>(a, un, 0), y1 = rb0.code + tile_row<kEpi>(a, un, 32);
+      const int64_t sy0 = rb0.scale + tile_row<kEpi>(a, un, 0), sy1 = rb0.scale + tile_row<kEpi>(a, un, 32);
+      const int it0 = it;
+      int cw = 0;
+      int sv[kTok];
+      for (int cx = 0; cx < L.nchunks && ok; ++cx) {
+        // weights up to `stages` chunks ahead of the activation rows
+        while (cw < L.nchunks && cw < cx + S) {
+          const int iw = it0 + cw, s = iw % S;
+          if (iw >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((iw / S) & 1) ^ 1, a.status))) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) stage_unit[s] = u;
+          const uint32_t st_base = sbase + s * L.stage_bytes;
+          const int k0 = cw * KC;
+          if (!stma) {
+            for (int w = lane; w < kRows * words; w += 32) {
+              const int r = w / words, cwd = w - r * words;
+              cp_async4(st_base + kScalesOff + r * kScaleRow + cwd * 4,
+                        a.scales + (rb0.scale + tile_row<kEpi>(a, un, r)) * (a.K / B) + k0 / B + cwd * 4);
+            }
+            cp_async_arrive(bar_full + 8 * s);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, wtx);
+          __syncwarp();
+          if (stma && lane == 0) {
+            const int32_t sx = k0 / (KC / kScaleRow);
+            tma_load_2d(st_base + kScalesOff, &smap, sx, static_cast<int32_t>(sy0), bar_full + 8 * s);
+            tma_load_2d(st_base + kScalesOff + 32 * kScaleRow, &smap, sx, static_cast<int32_t>(sy1), bar_full + 8 * s);
+          }
+          for (int q = lane; q < 2 * ncb; q += 32) {
+            const int rb = q & 1, cb = q >> 1;
+            tma_load_2d(st_base + (cb * kRows + rb * 32) * 128, &tmap, k0 / 2 + cb * 128,
+                        static_cast<int32_t>(rb ? y1 : y0), bar_full + 8 * s);
+          }
+          ++cw;
+        }
+        if (!ok) break;
+        if (!waited) {
+          pdl_wait();                 // x may come from the previous kernel
+          waited = true;
+          if (lane == 0) {
+            if (blockIdx.x == 0) *a.status = 0u;   // this call's status word
+            slot_begin(a.slot);
+          }
+        }
+        if (cx == 0) {
+          // per-token power-of-two scale: max|x_t| 2^-s in [2^14, 2^15), as x_to_f16_kernel
+          for (int i = 0; i < kTok; ++i) {
+            sv[i] = 0;
+            if (i >= un.ntok) continue;
+            const uint16_t* xr = a.x_bf16 + static_cast<int64_t>(un.slot0 + i) * a.K;
+            float amax = 0.f;
+            for (int h = lane * 8; h < a.K; h += 256) {
+              const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[j] << 16)), fabsf(__uint_as_float(w4[j] & 0xFFFF0000u))));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            int e2 = 0;
+            if (amax > 0.f && isfinite(amax)) {
+              int e;
+              frexpf(amax, &e);
+              e2 = (e - 1) - 14;
+            }
+            sv[i] = e2;
+            if (lane == 0) scl_w[un.slot0 + i] = ldexpf(1.0f, e2);
+          }
+        }
+        // the chunk's activation rows, f16, into the stage
+        const int s = (it0 + cx) % S;
+        uint8_t* xdst = smem + s * L.stage_bytes + kXOff;
+        for (int i = 0; i < un.ntok; ++i) {
+          const uint16_t* xr = a.x_bf16 + static_cast<int64_t>(un.slot0 + i) * a.K + cx * KC;
+          for (int h = lane * 8; h < KC; h += 256) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const __half lo = __float2half_rn(ldexpf(__uint_as_float(w4[j] << 16), -sv[i]));
+              const __half hi = __float2half_rn(ldexpf(__uint_as_float(w4[j] & 0xFFFF0000u), -sv[i]));
+              o4[j] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+            }
+            *reinterpret_cast<uint4*>(xdst + i * kXRow + h * 2) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full + 8 * s);
+      }
+      it = it0 + L.nchunks;
+    }
+    if (ok) {
+      // sentinel stage: no more work for this CTA (both arrivals)
+      const int s = it % S;
+      if (it < S || __all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / S) & 1) ^ 1, a.status))) {
+        if (lane == 0) {
+          stage_unit[s] = -1;
+          mbar_arrive(bar_full + 8 * s);
+          mbar_arrive(bar_full + 8 * s);
+        }
+        ++it;
+      }
+    }
+    if (!waited) {
+      pdl_wait();
+      if (lane == 0) {
+        if (blockIdx.x == 0) *a.status = 0u;
+        slot_begin(a.slot);
+      }
+    }
+    for (int d = 1; d <= S && d <= it; ++d) {
+      const int j = it - d;
+      mbar_wait(bar_full + 8 * (j % S), (j / S) & 1, a.status);
+    }
+    finish();
+    return;
+  }
 
   if (warp == kConsumers) {
     // ------------------------------- producer -------------------------------------
@@ -440,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
   // per-slot epilogue factors, loaded once so no unit's epilogue waits on global memory
   float* scl_s = reinterpret_cast<float*>(smem + L.scl_off);
-  if (L.scl_n > 0) {
+  if (L.scl_n > 0 && !fused_x) {      // (fused dense layer: the producer writes them)
     for (int i = threadIdx.x; i < L.scl_n; i += kConsumers * 32) {
       float v;
       if (kEpi == kEpiSwiglu) v = ldexpf(1.0f, a.sexp[perm_at(i) / a.topk]);

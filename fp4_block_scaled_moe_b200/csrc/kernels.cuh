@@ -100,7 +100,8 @@ struct DecodeArgs {
   const int64_t* row_off;
   const int64_t* srow_off;
   int64_t scale_rows_total;      // mixed-format buffers: rows of the scale buffer (else rows_total)
-  const __half* x16;             // activation rows, f16 [rows, K]
+  const __half* x16;             // activation rows, f16 [rows, K] (null: dense layer converting x_bf16)
+  const uint16_t* x_bf16;        // dense layer: bf16 x [T, K] when x16 is null
   const int* sexp;               // per token exponent (swiglu / linear) or null
   float limit;                   // swiglu clamp
   __half* h_out;                 // swiglu: [P, I]

@@ -539,9 +539,13 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   int* sexp = reinterpret_cast<int*>(ws + ctrl_bytes);
   __half* x16 = reinterpret_cast<__half*>(ws + ctrl_bytes + align_up(sizeof(int32_t) * T, kAlign));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, true,
-                     static_cast<const uint16_t*>(x_bf16), static_cast<int>(T), static_cast<int>(K), x16, sexp,
-                     ctrl));
+  // up to kRouteMaxPairs tokens the GEMV converts x itself in one launch (its per-token
+  // factors live in shared memory); beyond, x_to_f16_kernel converts it first
+  const bool fused = T <= kRouteMaxPairs;
+  if (!fused)
+    FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, true,
+                       static_cast<const uint16_t*>(x_bf16), static_cast<int>(T), static_cast<int>(K), x16, sexp,
+                       ctrl));
   DecodeArgs a{};
   a.fmt = fmt;
   a.epi = kEpiLinear;
@@ -556,8 +560,9 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   a.static_tiles = static_cast<int>(N / 64);
   a.e_begin = 0;
   a.e_end = 1;
-  a.x16 = x16;
-  a.sexp = sexp;
+  a.x16 = fused ? nullptr : x16;
+  a.x_bf16 = static_cast<const uint16_t*>(x_bf16);
+  a.sexp = fused ? nullptr : sexp;
   a.y_out = static_cast<uint16_t*>(y_bf16);
   a.ldo = static_cast<int>(N);
   a.status = &ctrl->status;
