@@ -272,8 +272,9 @@ def moe_fp4_expert_kernels(weights: MoEWeights, T: int, k: int) -> int:
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
-    """A 256-byte aligned device buffer (torch allocations are 512-byte aligned)."""
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    """A 256-byte aligned, zero-filled device buffer (torch allocations are 512-byte
+    aligned; zero-filled so that the control block's timing fields start valid)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def moe_fp4_forward(weights: MoEWeights, x, router_w, router_bias, k, workspace=None, route_out=None,

@@ -408,9 +408,15 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + (tmem_holder - sbase));
-  pdl_wait();
+  // The down GEMM's work units follow from the routing counts, which an earlier kernel
+  // (before gate_up) wrote, and its weights depend on nothing: its producer streams the
+  // first stages' weights before waiting for gate_up; only h (the B operand) waits.  Every
+  // other warp waits here.  gate_up needs the counts of the kernel just before it: it waits
+  // first.
+  const bool early_w = kEpi == kEpiDown;
+  if (!early_w || warp != 0) pdl_wait();
   pdl_launch_dependents();
-  if (threadIdx.x == 0) slot_begin(a.slot);
+  if (threadIdx.x == 0 && !early_w) slot_begin(a.slot);
 
   // per-expert unit prefix; units are ordered (expert, tile, token group)
   for (int e = threadIdx.x; e < E; e += kBsThreads) cnt[e] = a.counts[e];
@@ -456,6 +462,32 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     int it = 0;
     int u = blockIdx.x;
     bool ok = true;
+    // down: weights (A tile + its scale atom) of the first unit's first stages before the
+    // dependency wait; their stages get the rest (B tile + atoms) after it
+    int pre_n = 0;
+    if (early_w) {
+      if (u < n_units) {
+        const BsUnit un = bs_unit_of(u, cnt, off, pre, gpre, E, tiles, L.ntok_cap);
+        const int64_t rbase = static_cast<int64_t>(un.e - a.e_begin) * a.rows_per_expert;
+        const int64_t y0 = rbase + un.tile * 128, y1 = y0 + 64;
+        const uint8_t* sa = a.a_atoms + (static_cast<int64_t>(un.e - a.e_begin) * tiles + un.tile) * nk * 512;
+        const uint32_t sfb = 2 * un.ntok > 128 ? 1024u : 512u;
+        pre_n = min(S, nk);
+        for (int c = 0; c < pre_n; ++c) {
+          const uint32_t st = sbase + c * stg;
+          if (lane == 0) {
+            stage_unit[c] = u;
+            mbar_arrive_expect_tx(bar_full + 8 * c, static_cast<uint32_t>(128 * kKT / 2 + L.ncols * kKT) + 512u + sfb);
+            bulk_g2s(st + sf_off, sa + c * 512, 512, bar_full + 8 * c);
+            tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * c);
+            tma_load_2d(st + kATile / 2, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * c);
+          }
+          __syncwarp();
+        }
+      }
+      pdl_wait();
+      if (lane == 0) slot_begin(a.slot);
+    }
     while (ok) {
       if (u >= n_units) {
         const int s = it % S;
@@ -482,16 +514,19 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           ok = false;
           break;
         }
+        const bool a_done = it < pre_n;     // this stage's weights were issued before the wait
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st = sbase + s * stg;
         const uint32_t sf = st + sf_off;
         if (lane == 0) {
           const uint32_t sfb = two_b ? 1024u : 512u;
-          mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(128 * kKT / 2 + L.ncols * kKT) + 512u + sfb);
-          bulk_g2s(sf, sa + c * 512, 512, bar_full + 8 * s);
+          if (!a_done) {
+            mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(128 * kKT / 2 + L.ncols * kKT) + 512u + sfb);
+            bulk_g2s(sf, sa + c * 512, 512, bar_full + 8 * s);
+            tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * s);
+            tma_load_2d(st + kATile / 2, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
+          }
           bulk_g2s(sf + 512, sb + c * 1024, sfb, bar_full + 8 * s);
-          tma_load_2d(st, &tmA, c * kKT, static_cast<int32_t>(y0), bar_full + 8 * s);
-          tma_load_2d(st + kATile / 2, &tmA, c * kKT, static_cast<int32_t>(y1), bar_full + 8 * s);
           tma_load_2d(st + b_off, &tmB, c * kKT, brow0, bar_full + 8 * s);
         }
         __syncwarp();

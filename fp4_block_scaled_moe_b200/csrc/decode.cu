@@ -77,6 +77,7 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 
 struct Unit {
   int e, tile, slot0, ntok;
+  int ks;            // dense layer split over K: which share of the chunks (else 0)
 };
 
 // Exclusive scans by warp 0 over E experts: off = scan(cnt), pre = scan(units per expert),
@@ -132,14 +133,18 @@ __device__ __forceinline__ Unit unit_of(int u, const int* cnt, const int* off, c
   const int grp = local - un.tile * groups;
   un.slot0 = off[lo] + grp * kTok;
   un.ntok = min(kTok, n - grp * kTok);
+  un.ks = 0;
   return un;
 }
 
-__device__ __forceinline__ Unit unit_static(int u, int tiles, int T) {
+// dense layer: unit u -> {K share u % ksplit, tile, token group}
+__device__ __forceinline__ Unit unit_static(int u, int tiles, int T, int ksplit) {
   Unit un;
   un.e = 0;
-  un.tile = u % tiles;
-  un.slot0 = (u / tiles) * kTok;
+  un.ks = u % ksplit;
+  const int ub = u / ksplit;
+  un.tile = ub % tiles;
+  un.slot0 = (ub / tiles) * kTok;
   un.ntok = min(kTok, T - un.slot0);
   return un;
 }
@@ -201,6 +206,14 @@ __device__ __forceinline__ void cb4_lookup8(uint32_t w, const uint32_t (&lo)[4],
   }
 }
 
+// bf16x2 -> f16x2 of x 2^n with n split as two power-of-two factors f1 f2 (both exact
+// multiplications wherever the f16 result is not zero), rounded to nearest: the same bits as
+// converting ldexpf(x, n)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float f1, float f2) {
+  const __half2 h = __floats2half2_rn((__uint_as_float(w << 16) * f1) * f2, (__uint_as_float(w & 0xFFFF0000u) * f1) * f2);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <int kFmt, int kEpi, int kMode, int KC>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap smap,
@@ -229,8 +242,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   int* pre = reinterpret_cast<int*>(smem + L.pre_off);
   int* perm_s = reinterpret_cast<int*>(smem + L.perm_off);
 
-  // dense layer with bf16 x: the producer converts x itself (no separate launch) and streams
-  // the weights before waiting on the previous kernel (they do not depend on it)
+  // dense layer with bf16 x (no separate conversion launch): the producer streams the weights
+  // before waiting on the previous kernel (they do not depend on it) and the raw bf16 rows
+  // after it; the consumers convert the rows to f16 as they read them
   const bool fused_x = kMode == kModeStatic && a.x16 == nullptr;
   __shared__ unsigned int exit_count;
   if (threadIdx.x == 0) {
@@ -259,9 +273,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   };
 
   // ------------------------------- work units ---------------------------------------
+  // dense layer: the K chunks may be split over ksplit units (partial sums, reduced by a
+  // second kernel in a fixed order); nck chunks per unit
+  const int ksplit = (kMode == kModeStatic && a.ksplit > 1) ? a.ksplit : 1;
+  const int nck = L.nchunks / ksplit;
   int n_units;
   if (kMode == kModeStatic) {
-    n_units = tiles * ((a.T + kTok - 1) / kTok);
+    n_units = tiles * ((a.T + kTok - 1) / kTok) * ksplit;
   } else {
     const int E = a.E;
     if (kMode == kModeRoute) {
@@ -319,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     n_units = pre[E];
   }
   auto get_unit = [&](int u) -> Unit {
-    if (kMode == kModeStatic) return unit_static(u, tiles, a.T);
+    if (kMode == kModeStatic) return unit_static(u, tiles, a.T, ksplit);
     return unit_of(u, cnt, off, pre, a.E, tiles);
   };
   auto perm_at = [&](int slot) -> int {
@@ -338,7 +356,6 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
 
   if (kMode == kModeStatic && warp == kConsumers && fused_x) {
     // ------------------------- producer, dense layer with bf16 x ----------------------
-    float* scl_w = reinterpret_cast<float*>(smem + L.scl_off);
     const bool stma = a.scale_tma != 0;
     constexpr int words = kScaleRow / 4;
     const uint32_t wtx = static_cast<uint32_t>(kRows * (KC / 2) + (stma ? kRows * kScaleRow : 0));
@@ -352,10 +369,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
       const int64_t sy0 = rb0.scale + tile_row<kEpi>(a, un, 0), sy1 = rb0.scale + tile_row<kEpi>(a, un, 32);
       const int it0 = it;
       int cw = 0;
-      int sv[kTok];
-      for (int cx = 0; cx < L.nchunks && ok; ++cx) {
+      const int cb0 = un.ks * nck;               // first chunk of the unit's K share
+      for (int cx = 0; cx < nck && ok; ++cx) {
         // weights up to `stages` chunks ahead of the activation rows
-        while (cw < L.nchunks && cw < cx + S) {
+        while (cw < nck && cw < cx + S) {
           const int iw = it0 + cw, s = iw % S;
           if (iw >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((iw / S) & 1) ^ 1, a.status))) {
             ok = false;
@@ -363,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
           }
           if (lane == 0) stage_unit[s] = u;
           const uint32_t st_base = sbase + s * L.stage_bytes;
-          const int k0 = cw * KC;
+          const int k0 = (cb0 + cw) * KC;
           if (!stma) {
             for (int w = lane; w < kRows * words; w += 32) {
               const int r = w / words, cwd = w - r * words;
@@ -396,54 +413,16 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
             slot_begin(a.slot);
           }
         }
-        if (cx == 0) {
-          // per-token power-of-two scale: max|x_t| 2^-s in [2^14, 2^15), as x_to_f16_kernel
-          for (int i = 0; i < kTok; ++i) {
-            sv[i] = 0;
-            if (i >= un.ntok) continue;
-            const uint16_t* xr = a.x_bf16 + static_cast<int64_t>(un.slot0 + i) * a.K;
-            float amax = 0.f;
-            for (int h = lane * 8; h < a.K; h += 256) {
-              const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[j] << 16)), fabsf(__uint_as_float(w4[j] & 0xFFFF0000u))));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-            int e2 = 0;
-            if (amax > 0.f && isfinite(amax)) {
-              int e;
-              frexpf(amax, &e);
-              e2 = (e - 1) - 14;
-            }
-            sv[i] = e2;
-            if (lane == 0) scl_w[un.slot0 + i] = ldexpf(1.0f, e2);
-          }
-        }
-        // the chunk's activation rows, f16, into the stage
+        // the chunk's raw bf16 activation rows into the stage (the consumers convert them)
         const int s = (it0 + cx) % S;
-        uint8_t* xdst = smem + s * L.stage_bytes + kXOff;
-        for (int i = 0; i < un.ntok; ++i) {
-          const uint16_t* xr = a.x_bf16 + static_cast<int64_t>(un.slot0 + i) * a.K + cx * KC;
-          for (int h = lane * 8; h < KC; h += 256) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const __half lo = __float2half_rn(ldexpf(__uint_as_float(w4[j] << 16), -sv[i]));
-              const __half hi = __float2half_rn(ldexpf(__uint_as_float(w4[j] & 0xFFFF0000u), -sv[i]));
-              o4[j] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-            }
-            *reinterpret_cast<uint4*>(xdst + i * kXRow + h * 2) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-          }
-        }
+        if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(un.ntok * KC * 2));
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_full + 8 * s);
+        if (lane < un.ntok)
+          bulk_g2s(sbase + s * L.stage_bytes + kXOff + lane * kXRow,
+                   a.x_bf16 + static_cast<int64_t>(un.slot0 + lane) * a.K + (cb0 + cx) * KC,
+                   static_cast<uint32_t>(KC * 2), bar_full + 8 * s);
       }
-      it = it0 + L.nchunks;
+      it = it0 + nck;
     }
     if (ok) {
       // sentinel stage: no more work for this CTA (both arrivals)
@@ -477,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     int it = 0;
     bool ok = true;
     int u = blockIdx.x;
+    const bool stma = a.scale_tma != 0;   // the per-row scale bytes arrive as two TMA boxes
     while (true) {
       if (u >= n_units) {
         // sentinel stage: no more work for this CTA
@@ -497,12 +477,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
       const int64_t sy0 = rb0.scale + tile_row<kEpi>(a, un, 0), sy1 = rb0.scale + tile_row<kEpi>(a, un, 32);
       int xr = 0;
       if (lane < un.ntok) xr = (kEpi == kEpiSwiglu) ? perm_at(un.slot0 + lane) / a.topk : un.slot0 + lane;
-      const bool stma = a.scale_tma != 0;   // the per-row scale bytes arrive as two TMA boxes
       const uint32_t tx = static_cast<uint32_t>(kRows * (KC / 2) + un.ntok * KC * 2 +
                                                 ((kCb || stma) ? kRows * kScaleRow : 0) +
                                                 (kFmt == FP4_V2A ? kV2aLibBytes : 0));
       constexpr int words = kScaleRow / 4;
-      for (int c = 0; c < L.nchunks; ++c, ++it) {
+      for (int c = 0; c < nck; ++c, ++it) {
         const int s = it % L.stages;
         if (it >= L.stages &&
             !__all_sync(0xFFFFFFFFu, mbar_wait(bar_empty + 8 * s, ((it / L.stages) & 1) ^ 1, a.status))) {
@@ -511,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         }
         if (lane == 0) stage_unit[s] = u;
         const uint32_t st_base = sbase + s * L.stage_bytes;
-        const int k0 = c * KC;
+        const int k0 = (un.ks * nck + c) * KC;
         if (!kCb && !stma) {
           for (int w = lane; w < kRows * words; w += 32) {
             const int r = w / words, cw = w - r * words;
@@ -581,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
   const uint32_t x_off = kXOff + g * kXRow + t * 16 + jbase * 64;
   // per-slot epilogue factors, loaded once so no unit's epilogue waits on global memory
   float* scl_s = reinterpret_cast<float*>(smem + L.scl_off);
-  if (L.scl_n > 0 && !fused_x) {      // (fused dense layer: the producer writes them)
+  if (L.scl_n > 0 && !fused_x) {      // (fused dense layer: written at each unit's start)
     for (int i = threadIdx.x; i < L.scl_n; i += kConsumers * 32) {
       float v;
       if (kEpi == kEpiSwiglu) v = ldexpf(1.0f, a.sexp[perm_at(i) / a.topk]);
@@ -591,6 +570,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     }
     named_bar_sync();
   }
+  // fused dense layer: the stages hold raw bf16 rows, converted here to f16 x 2^-s_t with
+  // the per-token power of two of x_to_f16_kernel (max|x_t| 2^-s_t in [2^14, 2^15)), which
+  // each unit finds first (warp i scans token i of the unit)
+  __shared__ int xs_s[kTok];
+  if (fused_x) pdl_wait();
   int it = 0;
   while (true) {
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * (it % L.stages), (it / L.stages) & 1, a.status))) {
@@ -601,12 +585,42 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     if (u < 0) break;                              // sentinel: no more work
     const Unit un = get_unit(u);
     const float ts = (kFmt == FP4_NVFP4) ? a.tscale[un.e - a.e_begin] : 1.0f;   // used after the K loop
+    float xf1 = 1.0f, xf2 = 1.0f;                  // this thread's token (g): x16 = (x f1) f2
+    if (kMode == kModeStatic && fused_x) {
+      int sx = 0;
+      if (warp < un.ntok) {
+        const uint16_t* xr = a.x_bf16 + static_cast<int64_t>(un.slot0 + warp) * a.K;
+        float amax = 0.f;
+#pragma unroll 4
+        for (int h = lane * 8; h < a.K; h += 256) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xr + h);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[j] << 16)), fabsf(__uint_as_float(w4[j] & 0xFFFF0000u))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        if (amax > 0.f && isfinite(amax)) {
+          int e;
+          frexpf(amax, &e);
+          sx = (e - 1) - 14;
+        }
+        if (lane == 0) scl_s[un.slot0 + warp] = ldexpf(1.0f, sx);
+      }
+      if (lane == 0) xs_s[warp] = sx;
+      named_bar_sync();
+      const int n = -xs_s[g];                      // in [-113, 147] for finite bf16 rows
+      const int n1 = min(n, 127);
+      xf1 = __uint_as_float(static_cast<uint32_t>(n1 + 127) << 23);
+      xf2 = __uint_as_float(static_cast<uint32_t>(n - n1 + 127) << 23);
+    }
     float acc[2][4];
 #pragma unroll
     for (int m = 0; m < 2; ++m)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
-    for (int c = 0; c < L.nchunks; ++c, ++it) {
+    for (int c = 0; c < nck; ++c, ++it) {
       const int s = it % L.stages;
       if (c > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar_full + 8 * s, (it / L.stages) & 1, a.status))) {
         finish();
@@ -670,7 +684,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
 #pragma unroll
           for (int m = 0; m < 4; ++m) e2m1x8_to_f16x8(w[m], p[m][0], p[m][1], p[m][2], p[m][3]);
         }
-        const uint4 xq = *reinterpret_cast<const uint4*>(stp + x_off + jj * 64);
+        uint4 xq = *reinterpret_cast<const uint4*>(stp + x_off + jj * 64);
+        if (kMode == kModeStatic && fused_x)
+          xq = make_uint4(bf16x2_to_f16x2(xq.x, xf1, xf2), bf16x2_to_f16x2(xq.y, xf1, xf2),
+                          bf16x2_to_f16x2(xq.z, xf1, xf2), bf16x2_to_f16x2(xq.w, xf1, xf2));
         if (kCb) {
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt) {
@@ -766,8 +783,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
         const int r = idx & 63, i = idx >> 6;
         const float v = (L.scl_n > 0) ? (val(r, i) * ts) * scl_s[un.slot0 + i]
                                       : ldexpf(val(r, i) * ts, a.sexp[un.slot0 + i]);
-        a.y_out[static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        const int64_t o = static_cast<int64_t>(un.slot0 + i) * a.ldo + un.tile * kRows + r;
+        if (ksplit > 1) a.part[static_cast<int64_t>(un.ks) * a.T * a.ldo + o] = v;    // fp32 partial
+        else a.y_out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
     }
   }
@@ -839,10 +857,51 @@ fp4_status dispatch(const DecodeArgs& a, const Layout& L, const CUtensorMap& map
     return launch_one<kFmt, kEpiSwiglu, kModeRoute>(a, L, map, smap, grid, st, pdl);
   if (a.epi == kEpiSwiglu) return launch_one<kFmt, kEpiSwiglu, kModeList>(a, L, map, smap, grid, st, pdl);
   if (a.epi == kEpiDown) return launch_one<kFmt, kEpiDown, kModeList>(a, L, map, smap, grid, st, pdl);
-  return launch_one<kFmt, kEpiLinear, kModeStatic>(a, L, map, smap, grid, st, pdl);
+  if constexpr (kFmt == FP4_CB4 || kFmt == FP4_V2A) return FP4_ERR_UNSUPPORTED;   // (no dense layer)
+  else return launch_one<kFmt, kEpiLinear, kModeStatic>(a, L, map, smap, grid, st, pdl);
 }
 
 }  // namespace
+
+int linear_ksplit(int fmt, int64_t K, int64_t T, int64_t N, size_t part_bytes) {
+  if (K > INT32_MAX) return 1;
+  const Layout L = make_layout(fmt, static_cast<int>(K), 1, 0, 0);
+  if (L.kc == 0) return 1;
+  const int64_t base = (N / kRows) * ((T + kTok - 1) / kTok);
+  const int64_t slots = static_cast<int64_t>(ctas_per_sm(L.kc)) * num_sms();
+  int ks = 1;
+  while (L.nchunks % (2 * ks) == 0 && base * 2 * ks <= slots &&
+         static_cast<uint64_t>(2 * ks) * static_cast<uint64_t>(T) * static_cast<uint64_t>(N) * 4u <= part_bytes)
+    ks *= 2;
+  return ks;
+}
+
+// y = bf16 of the K shares' fp32 partial sums, added in share order (deterministic)
+__global__ void __launch_bounds__(256) linear_reduce_kernel(const float* __restrict__ part, int ksplit, int64_t n,
+                                                            uint16_t* __restrict__ y) {
+  // the next kernel on the stream may start now: what it reads before its own dependency
+  // wait (a layer's weights) does not depend on this one
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x * 4) {
+    float4 s = *reinterpret_cast<const float4*>(part + i);
+    for (int ks = 1; ks < ksplit; ++ks) {
+      const float4 v = *reinterpret_cast<const float4*>(part + ks * n + i);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(s.x)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(s.y))) << 16);
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(s.z)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(s.w))) << 16);
+    *reinterpret_cast<uint2*>(y + i) = make_uint2(lo, hi);
+  }
+}
+
+fp4_status launch_linear_reduce(const float* part, int ksplit, int64_t n_elems, uint16_t* y, cudaStream_t st) {
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n_elems / 4 + 255) / 256, num_sms() * 4)));
+  return launch_pdl(linear_reduce_kernel, dim3(grid), dim3(256), 0, st, true, part, ksplit, n_elems, y);
+}
 
 fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
   const int E = (a.mode == kModeStatic) ? 1 : a.E;
@@ -854,7 +913,8 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
   FP4_TRY(make_tmap_2d_u8(&map, a.codes, static_cast<uint64_t>(a.K / 2), static_cast<uint64_t>(a.rows_total),
                           static_cast<uint64_t>(a.K / 2), 128, 32, CU_TENSOR_MAP_SWIZZLE_128B));
   int grid = ctas_per_sm(L.kc) * num_sms();
-  if (a.mode == kModeStatic) grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok));
+  if (a.mode == kModeStatic)
+    grid = std::min(grid, a.static_tiles * ((a.T + kTok - 1) / kTok) * std::max(1, a.ksplit));
   // the per-row scale bytes (E2M1 block scales, CB4 codebooks, V2a group records) by TMA
   // when a stage's share of a row and the row stride are multiples of 16 bytes
   DecodeArgs b = a;
@@ -876,16 +936,26 @@ fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl) {
 // y[t, n] = bf16( sum_{j = 0..k-1} o[inv[t k + j], n] ), fixed j order (deterministic).
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv,
                                                       int T, int k, int H, uint16_t* __restrict__ y) {
+  pdl_launch_dependents();    // (the next layer's router weights do not depend on this kernel)
   pdl_wait();
   const int64_t n4 = static_cast<int64_t>(T) * (H / 4);
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int tt = static_cast<int>(i / (H / 4));
     const int h = static_cast<int>(i % (H / 4)) * 4;
+    // the k slot rows are fetched together (eight at a time) and summed in j order
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(o + static_cast<int64_t>(inv[tt * k + j]) * H + h);
-      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int r[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) r[j] = (j0 + j < k) ? inv[tt * k + j0 + j] : -1;
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (r[j] >= 0) v[j] = *reinterpret_cast<const float4*>(o + static_cast<int64_t>(r[j]) * H + h);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (r[j] >= 0) { s.x += v[j].x; s.y += v[j].y; s.z += v[j].z; s.w += v[j].w; }
     }
     const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(s.x)) |
                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(s.y))) << 16);
@@ -893,7 +963,6 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(s.w))) << 16);
     *reinterpret_cast<uint2*>(y + static_cast<int64_t>(tt) * H + h) = make_uint2(lo, hi);
   }
-  pdl_launch_dependents();
 }
 
 // Expert-parallel partial sum: only the slots of this call's experts contribute, fp32 out.
@@ -908,11 +977,23 @@ __global__ void __launch_bounds__(256) combine_partial_kernel(const float* __res
     const int tt = static_cast<int>(i / (H / 4));
     const int h = static_cast<int>(i % (H / 4)) * 4;
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const int e = ids[tt * k + j];
-      if (e < e_begin || e >= e_end) continue;
-      const float4 v = *reinterpret_cast<const float4*>(o + static_cast<int64_t>(inv[tt * k + j]) * H + h);
-      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int r[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        r[j] = -1;
+        if (j0 + j < k) {
+          const int e = ids[tt * k + j0 + j];
+          if (e >= e_begin && e < e_end) r[j] = inv[tt * k + j0 + j];
+        }
+      }
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (r[j] >= 0) v[j] = *reinterpret_cast<const float4*>(o + static_cast<int64_t>(r[j]) * H + h);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (r[j] >= 0) { s.x += v[j].x; s.y += v[j].y; s.z += v[j].z; s.w += v[j].w; }
     }
     *reinterpret_cast<float4*>(y + static_cast<int64_t>(tt) * H + h) = s;
   }

@@ -111,9 +111,16 @@ struct DecodeArgs {
   uint32_t* status;
   KernelSlot* slot;              // per-launch device timing (or null)
   uint32_t* unit_next;           // dynamic scheduling counter (zeroed by the router), or null
+  int ksplit;                    // linear: units per 64-row tile and token group along K (0, 1: none)
+  float* part;                   // linear with ksplit > 1: fp32 partial sums [ksplit][T][N]
 };
 
 fp4_status launch_decode(const DecodeArgs& a, cudaStream_t st, bool pdl);
+// Dense layer: how many K shares (a power of two dividing the stage count) keep the
+// layer's units within one wave of CTAs while [ks][T][N] fp32 partials fit part_bytes
+int linear_ksplit(int fmt, int64_t K, int64_t T, int64_t N, size_t part_bytes);
+// y[t, n] = bf16( sum over ks = 0, 1, ... of part[ks][t][n] ), n_elems = T N (multiple of 4)
+fp4_status launch_linear_reduce(const float* part, int ksplit, int64_t n_elems, uint16_t* y, cudaStream_t st);
 
 // The bf16 experts of a mixed-format fused buffer (dense16.cu): same units and epilogues
 // as the grouped GEMV; weights at weights + offset[e - e_begin], bf16 rows of K.

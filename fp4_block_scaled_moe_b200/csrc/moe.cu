@@ -509,10 +509,13 @@ extern "C" fp4_status fp4_f32_to_bf16(const float* in, int64_t n, void* out, voi
   return launch_f32_to_bf16(in, n, static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream));
 }
 
+// fp32 partial sums of a dense layer split over K (few tokens, few output tiles)
+constexpr size_t kLinearPartBytes = size_t(1) << 20;
+
 extern "C" size_t fp4_linear_workspace_size(int32_t T, int64_t K) {
   if (T <= 0 || K <= 0) return 0;
   return align_up(sizeof(WsControl), kAlign) + align_up(sizeof(int32_t) * T, kAlign) +
-         align_up(sizeof(uint16_t) * static_cast<size_t>(T) * static_cast<size_t>(K), kAlign);
+         align_up(sizeof(uint16_t) * static_cast<size_t>(T) * static_cast<size_t>(K), kAlign) + kLinearPartBytes;
 }
 
 extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K,
@@ -538,10 +541,13 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   const size_t ctrl_bytes = align_up(sizeof(WsControl), kAlign);
   int* sexp = reinterpret_cast<int*>(ws + ctrl_bytes);
   __half* x16 = reinterpret_cast<__half*>(ws + ctrl_bytes + align_up(sizeof(int32_t) * T, kAlign));
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(x16) +
+                                         align_up(sizeof(uint16_t) * static_cast<size_t>(T) * static_cast<size_t>(K), kAlign));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // up to kRouteMaxPairs tokens the GEMV converts x itself in one launch (its per-token
-  // factors live in shared memory); beyond, x_to_f16_kernel converts it first
-  const bool fused = T <= kRouteMaxPairs;
+  // up to kLinearFusedTokens tokens the GEMV converts x itself in one launch (each work unit
+  // scans its 8 token rows for their scale first); beyond, x_to_f16_kernel converts it once
+  constexpr int64_t kLinearFusedTokens = 64;
+  const bool fused = T <= kLinearFusedTokens;
   if (!fused)
     FP4_TRY(launch_pdl(x_to_f16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, true,
                        static_cast<const uint16_t*>(x_bf16), static_cast<int>(T), static_cast<int>(K), x16, sexp,
@@ -567,5 +573,10 @@ extern "C" fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, 
   a.ldo = static_cast<int>(N);
   a.status = &ctrl->status;
   a.slot = &ctrl->slot[0];
-  return launch_decode(a, st, true);
+  // too few 64-row tiles x token groups to fill the GPU: split K, partials reduced after
+  a.ksplit = linear_ksplit(fmt, K, T, N, kLinearPartBytes);
+  a.part = part;
+  FP4_TRY(launch_decode(a, st, true));
+  if (a.ksplit > 1) FP4_TRY(launch_linear_reduce(part, a.ksplit, T * N, static_cast<uint16_t*>(y_bf16), st));
+  return FP4_OK;
 }

@@ -16,6 +16,11 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// The logit of an order key (inverse of order_key for every number; a NaN key reads as a NaN)
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // Top-k of one token's logits by one warp (E <= 1024, k <= 32): descending logit, ties to
 // the lower expert.  Writes ids[0..k) and, when gw != null, the softmax over the k logits.
 template <int kPer>
@@ -51,7 +56,7 @@ __device__ __forceinline__ void topk_warp_n(const float* __restrict__ lg, int E,
       if (ob > best || (ob == best && oe < best_e)) { best = ob; best_e = oe; }
     }
     if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
-    const float l = lg[best_e];
+    const float l = key_value(best);                 // the logit itself (-0 read as +0)
     if (r == 0) m = l;
     const float z = expf(l - m);
     sum += z;

@@ -369,11 +369,16 @@ fp4_status fp4_f32_to_bf16(const float* in, int64_t n, void* out, void* stream);
  * W4A16_NVFP4).  workspace: at least fp4_linear_workspace_size(T, K) bytes, 256-byte
  * aligned; its first 256 bytes are a control block like moe_fp4_forward's, read by
  * fp4_workspace_status and by fp4_workspace_kernel_stats (gate_up_* = the linear kernel).
- * Up to 1024 tokens the call is one kernel: it starts streaming the weights before it waits
- * for the previous kernel on the stream (so consecutive layers overlap), and reads x and
- * writes y only after that wait.  The weights must therefore be complete when the call is
- * made (not written by a kernel that is still running on the stream and lets dependents
- * start early); this library's packers finish before any later kernel starts.
+ * Up to 64 tokens the GEMV converts x itself (no separate conversion launch): it starts
+ * streaming the weights before it waits for the previous kernel on the stream (so
+ * consecutive layers overlap), and reads x and writes y only after that wait.  The
+ * weights must therefore be complete when the call is made (not written by a kernel that
+ * is still running on the stream and lets dependents start early); this library's packers
+ * finish before any later kernel starts.  When the layer has too few 64-row tiles x
+ * 8-token groups to fill the GPU, K is split over several CTAs and a second small kernel
+ * adds their fp32 partial sums in a fixed order (y stays deterministic).  The timing
+ * fields of the control block start valid when the workspace was zero-filled before its
+ * first use (the Python binding's workspaces are).
  */
 size_t fp4_linear_workspace_size(int32_t T, int64_t K);
 fp4_status fp4_linear(fp4_format fmt, const void* x_bf16, int32_t T, int64_t K, const uint8_t* codes,

@@ -65,3 +65,47 @@ def test_repeat_and_graph_replay_bit_identical(name, cfg, variant, prepared):
         assert torch.equal(b1, yg.view(torch.int16)), "graph replay differs"
     assert api.fp4_workspace_status(ws1) == "FP4_OK"
     del g
+
+
+_LINEAR = [
+    ("c1_full_split", C.LINEAR_C1),                                               # one launch + K shares
+    ("nvfp4_t48_split2", C.LinearConfig("linear_nvfp4_t48", "nvfp4", 48, 1024, 2048)),
+    ("mxfp4_t200", C.LinearConfig("linear_mxfp4_t200", "mxfp4", 200, 512, 1024)),   # separate x conversion
+]
+
+
+@pytest.mark.parametrize("name,cfg", _LINEAR, ids=[c[0] for c in _LINEAR])
+def test_linear_repeat_and_graph_replay_bit_identical(name, cfg):
+    """The dense layer likewise: its K shares are added in a fixed order by the reduce."""
+    from fp4_block_scaled_moe_b200 import api, fp4_linear, fp4_pack
+    from synth import draws as D
+    w = D.expert_weights(cfg.seed, C.TID_LINEAR, (cfg.N, cfg.K), sigma=cfg.sigma)
+    x_bits = D.activations_bf16(cfg.seed, cfg.T, cfg.K)
+    c, s_, t = fp4_pack(torch.from_numpy(w).cuda(), cfg.fmt)
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    nbytes = int(api.L.load().fp4_linear_workspace_size(cfg.T, cfg.K))
+    ws1 = api.alloc_workspace(nbytes, x.device)
+    ws2 = api.alloc_workspace(nbytes + 4096, x.device)
+    y1 = fp4_linear(x, c, s_, t, cfg.fmt, workspace=ws1)
+    y2 = fp4_linear(x, c, s_, t, cfg.fmt, workspace=ws1)
+    y3 = fp4_linear(x, c, s_, t, cfg.fmt, workspace=ws2)
+    torch.cuda.synchronize()
+    b1 = y1.view(torch.int16)
+    assert torch.equal(b1, y2.view(torch.int16))
+    assert torch.equal(b1, y3.view(torch.int16))
+    yg = torch.empty_like(y1)
+    st = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        fp4_linear(x, c, s_, t, cfg.fmt, workspace=ws1, y=yg)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=st):
+            fp4_linear(x, c, s_, t, cfg.fmt, workspace=ws1, y=yg)
+    for _ in range(3):
+        yg.fill_(float("nan"))
+        with torch.cuda.stream(st):
+            g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(b1, yg.view(torch.int16))
+    assert api.fp4_workspace_status(ws1) == "FP4_OK"
+    del g

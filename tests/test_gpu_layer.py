@@ -29,9 +29,13 @@ def _y_host(y):
     return D.bf16_bits_to_f32(y.view(torch.int16).cpu().numpy().view(np.uint16)).reshape(y.shape)
 
 
+# up to 64 tokens the dense layer is one kernel that converts x itself; above, x is
+# converted by a separate launch first (the many-token cases)
 @pytest.mark.parametrize("cfg", [C.small(C.LINEAR_C1), C.LINEAR_C1,
-                                 C.small(C.LinearConfig("linear_nvfp4", "nvfp4", 16, 2048, 2048))],
-                         ids=["c1_small", "c1_full", "nvfp4_small"])
+                                 C.small(C.LinearConfig("linear_nvfp4", "nvfp4", 16, 2048, 2048)),
+                                 C.LinearConfig("linear_mxfp4_many_tokens", "mxfp4", 1100, 128, 512),
+                                 C.LinearConfig("linear_nvfp4_many_tokens", "nvfp4", 1030, 192, 768)],
+                         ids=["c1_small", "c1_full", "nvfp4_small", "mxfp4_many_tokens", "nvfp4_many_tokens"])
 def test_linear(cfg):
     from fp4_block_scaled_moe_b200 import fp4_linear, fp4_pack
     w = D.expert_weights(cfg.seed, C.TID_LINEAR, (cfg.N, cfg.K), sigma=cfg.sigma)
@@ -45,6 +49,42 @@ def test_linear(cfg):
         deq = F.nvfp4_dequantize(*F.nvfp4_quantize(w))
     ref = M.linear(D.bf16_bits_to_f32(x_bits), deq)
     check_tolerance(_y_host(y), ref)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_linear_fused_conversion_bits(fmt):
+    """The one-launch dense layer (64 tokens) converts x to f16 inside the GEMV; the
+    two-launch one (65 tokens) converts it in a separate kernel first.  A token's output
+    does not depend on the other tokens, so the first 64 rows of both calls agree bit for
+    bit -- over rows whose power-of-two scale spans the whole bf16 range: a zero row, rows
+    of subnormal size (scale factor above 2^127), rows near the bf16 maximum."""
+    from fp4_block_scaled_moe_b200 import fp4_linear, fp4_pack
+    K, N = 1024, 192
+    w = D.expert_weights(11, C.TID_LINEAR, (N, K), sigma=0.02)
+    x = D.bf16_bits_to_f32(D.activations_bf16(11, 65, K)).astype(np.float32)
+    exps = np.arange(65) % 41 - 20
+    exps[3], exps[5], exps[9], exps[17] = -128, -131, 100, 110
+    x = np.ldexp(x, exps[:, None]).astype(np.float32)
+    x[7] = 0.0
+    x_bits = D.f32_to_bf16_bits(x)
+    c, s, t = fp4_pack(torch.from_numpy(w).cuda(), fmt)
+    xd = _bf16_dev(x_bits)
+    y65 = fp4_linear(xd, c, s, t, fmt)
+    y64 = fp4_linear(xd[:64].contiguous(), c, s, t, fmt)
+    torch.cuda.synchronize()
+    assert torch.equal(y64.view(torch.int16), y65[:64].view(torch.int16))
+    if fmt == "mxfp4":
+        deq = F.mxfp4_dequantize(*F.mxfp4_quantize(w))
+    else:
+        deq = F.nvfp4_dequantize(*F.nvfp4_quantize(w))
+    ref = M.linear(D.bf16_bits_to_f32(x_bits), deq)
+    got = _y_host(y65)
+    for r in range(65):          # each row against its own magnitude (normal bf16 outputs)
+        scale = float(np.max(np.abs(ref[r])))
+        if scale > 2.0 ** -100:
+            check_tolerance(got[r] / scale, ref[r] / scale)
+        else:
+            assert np.all(np.abs(got[r]) <= 2.0 ** -100)
 
 
 def check_selection(lg, gids, k):
