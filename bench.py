@@ -522,6 +522,10 @@ def moe_roofline(cfg, counts, extra_gu, kern_ms, tensor, peaks):
     _, gu_per_expert = per_expert_bytes(cfg)
     d = int(np.count_nonzero(counts))
     P = cfg.T * cfg.k
+    if cfg.fmt == "mixed":
+        # the GEMV reads the routed MXFP4 experts only (the bf16 ones run in dense16_kernel)
+        d -= sum(1 for e in cfg.bf16_experts if counts[e] > 0)
+        extra_gu = None
     alg = d * gu_per_expert + cfg.T * cfg.H * 2 + P * cfg.I * 2
     if extra_gu is not None:
         alg += int(np.sum(extra_gu[counts > 0]))

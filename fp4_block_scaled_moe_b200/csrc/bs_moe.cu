@@ -136,12 +136,14 @@ __device__ __forceinline__ void warp_split2(float v, uint32_t& q1, uint32_t& q2,
   s2 = static_cast<uint32_t>(e2 + 127);
 }
 
-// One 32-element block of token row t (bf16) -> its two E4M3 terms in rows 2 slot and
-// 2 slot + 1 of q, and the two UE8M0 scales into the token group's atoms (row 2i, 2i+1).
-__device__ __forceinline__ void split_block(const uint16_t* __restrict__ x, int t, int slot, int b, int i,
-                                            int64_t gid, int H, uint8_t* __restrict__ q,
-                                            uint8_t* __restrict__ atoms) {
-  const int kb128 = H / 128;
+// The two E4M3 terms of one 32-element block of a token row and their UE8M0 scales
+struct Split32 {
+  uint32_t w1[8], w2[8];
+  int e1, e2;
+};
+
+// One 32-element block b of token row t (bf16) -> its two-term split
+__device__ __forceinline__ void split_compute(const uint16_t* __restrict__ x, int t, int b, int H, Split32& sp) {
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + 32 * b);
   float v[32];
 #pragma unroll
@@ -159,7 +161,8 @@ __device__ __forceinline__ void split_block(const uint16_t* __restrict__ x, int 
   for (int ii = 0; ii < 32; ++ii) amax = fmaxf(amax, fabsf(v[ii]));
   const int e1 = e4m3_block_exp(amax);
   const float inv1 = exp2i(-e1), up1 = exp2i(e1);
-  uint32_t w1[8], w2[8];
+  uint32_t* w1 = sp.w1;
+  uint32_t* w2 = sp.w2;
   float ramax = 0.f;
 #pragma unroll
   for (int ii = 0; ii < 32; ++ii) {
@@ -179,22 +182,47 @@ __device__ __forceinline__ void split_block(const uint16_t* __restrict__ x, int 
     if ((ii & 3) == 0) w2[ii >> 2] = 0;
     w2[ii >> 2] |= c << (8 * (ii & 3));
   }
+  sp.e1 = e1;
+  sp.e2 = e2;
+}
+
+// A block's split into rows 2 slot and 2 slot + 1 of q, and its two UE8M0 scales into the
+// token group's atoms (rows 2i, 2i + 1)
+__device__ __forceinline__ void split_store(const Split32& sp, int slot, int b, int i, int64_t gid, int H,
+                                            uint8_t* __restrict__ q, uint8_t* __restrict__ atoms) {
+  const int kb128 = H / 128;
   uint4* d1 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot)) * H + 32 * b);
   uint4* d2 = reinterpret_cast<uint4*>(q + (2 * static_cast<int64_t>(slot) + 1) * H + 32 * b);
-  d1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-  d1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
-  d2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-  d2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+  d1[0] = make_uint4(sp.w1[0], sp.w1[1], sp.w1[2], sp.w1[3]);
+  d1[1] = make_uint4(sp.w1[4], sp.w1[5], sp.w1[6], sp.w1[7]);
+  d2[0] = make_uint4(sp.w2[0], sp.w2[1], sp.w2[2], sp.w2[3]);
+  d2[1] = make_uint4(sp.w2[4], sp.w2[5], sp.w2[6], sp.w2[7]);
   uint8_t* at = atoms + (gid * kb128 + (b >> 2)) * 1024 + (b & 3);
-  at[sf_row_off2(2 * i)] = static_cast<uint8_t>(e1 + 127);
-  at[sf_row_off2(2 * i + 1)] = static_cast<uint8_t>(e2 + 127);
+  at[sf_row_off2(2 * i)] = static_cast<uint8_t>(sp.e1 + 127);
+  at[sf_row_off2(2 * i + 1)] = static_cast<uint8_t>(sp.e2 + 127);
+}
+
+// Expert of a slot (largest e with off[e] <= slot), its position in the expert's token
+// group and the group's number across experts
+__device__ __forceinline__ void slot_place(const int* off, const int* gpre, int E, int cap, int slot, int& i,
+                                           int64_t& gid) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= slot) lo = mid; else hi = mid - 1;
+  }
+  const int local = slot - off[lo];
+  const int grp = local / cap;
+  i = local - grp * cap;
+  gid = static_cast<int64_t>(gpre[lo]) + grp;
 }
 
 // x [T][H] bf16 -> slot-ordered two-term MXFP8 rows q [2P][H] E4M3 (rows 2i, 2i + 1 for
 // slot i = token perm[i] / k) and their UE8M0 scales as token-group atoms.  One thread
-// per 32-element block.
+// per 32-element block of a token: the split is computed once and stored into each of the
+// token's k slots (inv: pair -> slot).
 __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict__ x,
-                                                      const int32_t* __restrict__ perm,
+                                                      const int32_t* __restrict__ inv,
                                                       const int32_t* __restrict__ counts,
                                                       const int32_t* __restrict__ offsets, int E, int k, int P,
                                                       int H, int cap, uint8_t* __restrict__ q,
@@ -223,19 +251,19 @@ __global__ void __launch_bounds__(256) split_x_kernel(const uint16_t* __restrict
   for (int e = threadIdx.x; e <= E; e += blockDim.x) off_s[e] = offsets[e];
   __syncthreads();
   const int nb = H / 32;
-  const int64_t total = static_cast<int64_t>(P) * nb;
+  const int64_t total = static_cast<int64_t>(P / k) * nb;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int slot = static_cast<int>(idx / nb), b = static_cast<int>(idx % nb);
-    int lo = 0, hi = E - 1;                    // expert of the slot: largest e with off[e] <= slot
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (off_s[mid] <= slot) lo = mid; else hi = mid - 1;
+    const int t = static_cast<int>(idx / nb), b = static_cast<int>(idx % nb);
+    Split32 sp;
+    split_compute(x, t, b, H, sp);
+    for (int j = 0; j < k; ++j) {
+      const int slot = inv[t * k + j];
+      int i;
+      int64_t gid;
+      slot_place(off_s, gpre_s, E, cap, slot, i, gid);
+      split_store(sp, slot, b, i, gid, H, q, atoms);
     }
-    const int local = slot - off_s[lo];
-    const int grp = local / cap, i = local - grp * cap;
-    const int64_t gid = gpre_s[lo] + grp;
-    split_block(x, perm[slot] / k, slot, b, i, gid, H, q, atoms);
   }
   pdl_launch_dependents();
 }
@@ -315,19 +343,19 @@ __global__ void __launch_bounds__(512) route_split_kernel(
       if (e < E) counts[e] = cnt[e];
       offsets[e] = off[e];
     }
+  // one thread per (slot, 32-block): at decode sizes the parallelism matters more than the
+  // repeated split of a token's blocks
   const int nb = H / 32;
   const int64_t total = static_cast<int64_t>(P) * nb;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int slot = static_cast<int>(idx / nb), b = static_cast<int>(idx % nb);
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (off[mid] <= slot) lo = mid; else hi = mid - 1;
-    }
-    const int local = slot - off[lo];
-    const int grp = local / cap, i = local - grp * cap;
-    split_block(x, perm_s[slot] / k, slot, b, i, static_cast<int64_t>(gpre[lo]) + grp, H, q, atoms);
+    Split32 sp;
+    split_compute(x, perm_s[slot] / k, b, H, sp);
+    int i;
+    int64_t gid;
+    slot_place(off, gpre, E, cap, slot, i, gid);
+    split_store(sp, slot, b, i, gid, H, q, atoms);
   }
   pdl_launch_dependents();
 }
@@ -733,11 +761,11 @@ bool bs_layout(int T, int E, BsLayout* L) {
 
 }  // namespace
 
-fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t* counts, const int32_t* offsets,
+fp4_status launch_split_x(const uint16_t* x, const int32_t* inv, const int32_t* counts, const int32_t* offsets,
                           int E, int k, int P, int H, int ntok_cap, uint8_t* q, uint8_t* atoms, cudaStream_t st) {
-  const int64_t total = static_cast<int64_t>(P) * (H / 32);
+  const int64_t total = static_cast<int64_t>(P / k) * (H / 32);
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, num_sms() * 16)));
-  return launch_pdl(split_x_kernel, dim3(grid), dim3(256), 0, st, true, x, perm, counts, offsets, E, k, P, H,
+  return launch_pdl(split_x_kernel, dim3(grid), dim3(256), 0, st, true, x, inv, counts, offsets, E, k, P, H,
                     ntok_cap, q, atoms);
 }
 

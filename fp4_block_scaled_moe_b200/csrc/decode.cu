@@ -191,13 +191,16 @@ __device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel
 
 __device__ __forceinline__ void cb4_lookup8(uint32_t w, const uint32_t (&lo)[4], const uint32_t (&hi)[4],
                                             uint32_t (&h)[4]) {
+  // bit 3 of every index at a byte's top bit: even nibbles in w << 4, odd ones in w; one
+  // sign-replicating byte-permute per half turns them into the select masks (byte i =
+  // 0xFF where index i of the half is >= 8)
+  const uint32_t ws = w << 4;
+  const uint32_t msks[2] = {prmt_sx(ws, w, 0xD9C8u), prmt_sx(ws, w, 0xFBEAu)};
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    const uint32_t v = half ? (w >> 16) : (w & 0xFFFFu);
+    const uint32_t v = half ? (w >> 16) : w;
     const uint32_t sel = v & 0x7777u;
-    const uint32_t r = __byte_perm(v, 0u, 0x1100);                  // bytes B0 B0 B1 B1
-    const uint32_t sgn = (r & 0xFF00FF00u) | ((r << 4) & 0x00FF00FFu);   // bit 3 of nibble i -> bit 7 of byte i
-    const uint32_t msk = prmt_sx(sgn, 0u, 0xBA98u);                 // byte i = 0xFF where index i >= 8
+    const uint32_t msk = msks[half];
     const uint32_t la = __byte_perm(lo[0], lo[1], sel), lb = __byte_perm(lo[2], lo[3], sel);
     const uint32_t ha = __byte_perm(hi[0], hi[1], sel), hb = __byte_perm(hi[2], hi[3], sel);
     const uint32_t L = (la & ~msk) | (lb & msk), H = (ha & ~msk) | (hb & msk);
@@ -751,12 +754,27 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KC))
     };
     // ---- fused epilogue ----
     // CB4 sparse term of row r against an activation row (same scaling as the MMA input)
+    // (four outliers at a time: their columns and values, then the activations, are loaded
+    // together; the products are added in ascending position order)
     auto sparse = [&](int r, const __half* xrow) -> float {
       if (!kCb || a.sp_rowptr == nullptr) return 0.f;
       const int64_t R = unit_row<kEpi>(a, un, r);
+      const int j1 = a.sp_rowptr[R + 1];
       float acc_s = 0.f;
-      for (int j = a.sp_rowptr[R]; j < a.sp_rowptr[R + 1]; ++j)
-        acc_s = fmaf(__half2float(__ushort_as_half(a.sp_val[j])), __half2float(xrow[a.sp_col[j]]), acc_s);
+      for (int j = a.sp_rowptr[R]; j < j1; j += 4) {
+        int c[4];
+        float v[4], xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          c[q] = (j + q < j1) ? a.sp_col[j + q] : 0;
+          v[q] = (j + q < j1) ? __half2float(__ushort_as_half(a.sp_val[j + q])) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = __half2float(xrow[c[q]]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (j + q < j1) acc_s = fmaf(v[q], xv[q], acc_s);
+      }
       return acc_s;
     };
     if (kEpi == kEpiSwiglu) {

@@ -9,10 +9,10 @@
 // the same epilogues (SwiGLU with its clamp into f16 h, or the gate-weighted fp32 output
 // in slot order), so the combine sums both kinds alike.
 //
-// One CTA per unit at a time (8 warps, 8 rows each): a warp streams its row's bf16 weights
-// 16 bytes per lane and multiplies them with the unit's f16 activation rows in fp32; the
-// lanes' partial sums meet in a fixed butterfly order (deterministic).  These experts are
-// the few a checkpoint excludes, so the kernel favours simplicity over peak bandwidth.
+// One CTA per unit at a time (8 warps, 8 rows each): a warp streams four of its rows' bf16
+// weights at a time, 16 bytes per lane and two K chunks ahead (eight loads in flight per
+// lane), and multiplies them with the unit's f16 activation rows in fp32; the lanes'
+// partial sums meet in a fixed butterfly order (deterministic).
 #include "kernels.cuh"
 
 namespace fp4 {
@@ -28,7 +28,7 @@ __device__ __forceinline__ bool d16_mine(const Dense16Args& a, int e) {
 }
 
 template <int kEpi>
-__global__ void __launch_bounds__(kD16Threads) dense16_kernel(const Dense16Args a) {
+__global__ void __launch_bounds__(kD16Threads, 1) dense16_kernel(const Dense16Args a) {
   __shared__ int cnt[kD16MaxE + 1], off[kD16MaxE + 1], pre[kD16MaxE + 1];
   __shared__ float red[kD16Rows][kD16Tok];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -62,46 +62,76 @@ __global__ void __launch_bounds__(kD16Threads) dense16_kernel(const Dense16Args 
     const int tile = local / groups, grp = local - tile * groups;
     const int slot0 = off[e] + grp * kD16Tok, ntok = min(kD16Tok, n - grp * kD16Tok);
     const uint8_t* wbase = a.weights + a.offset[e - a.e_begin];
-    for (int rr = 0; rr < kD16Rows / 8; ++rr) {
-      const int r = warp * (kD16Rows / 8) + rr;    // row of the unit
-      const int64_t row = (kEpi == kEpiSwiglu) ? (r < 32 ? tile * 32 + r : a.inter + tile * 32 + (r - 32))
-                                               : static_cast<int64_t>(tile) * kD16Rows + r;
-      const uint16_t* wrow = reinterpret_cast<const uint16_t*>(wbase) + row * a.K;
-      float acc[kD16Tok];
+    int64_t xr[kD16Tok];                         // activation row of each token of the unit
 #pragma unroll
-      for (int i = 0; i < kD16Tok; ++i) acc[i] = 0.f;
-      for (int k = lane * 8; k < a.K; k += 256) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(wrow + k);
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-        float wf[8];
+    for (int i = 0; i < kD16Tok; ++i) {
+      const int slot = slot0 + min(i, ntok - 1);
+      xr[i] = (kEpi == kEpiSwiglu) ? a.perm[slot] / a.topk : slot;
+    }
+    // a warp's 8 rows in two groups of four; each step keeps 2 K chunks x 4 rows of weights
+    // (eight 16-byte loads per lane) in flight
+    for (int rg = 0; rg < 2; ++rg) {
+      const uint16_t* wrow[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          wf[2 * j] = __uint_as_float(ww[j] << 16);
-          wf[2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int r = warp * (kD16Rows / 8) + rg * 4 + q;   // row of the unit
+        const int64_t row = (kEpi == kEpiSwiglu) ? (r < 32 ? tile * 32 + r : a.inter + tile * 32 + (r - 32))
+                                                 : static_cast<int64_t>(tile) * kD16Rows + r;
+        wrow[q] = reinterpret_cast<const uint16_t*>(wbase) + row * a.K;
+      }
+      float acc[4][kD16Tok];
 #pragma unroll
-        for (int i = 0; i < kD16Tok; ++i) {
-          if (i >= ntok) break;
-          const int slot = slot0 + i;
-          const int64_t xr = (kEpi == kEpiSwiglu) ? a.perm[slot] / a.topk : slot;
-          const uint4 xv = *reinterpret_cast<const uint4*>(a.x16 + xr * a.K + k);
-          const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&xx[j]));
-            acc[i] = fmaf(wf[2 * j], xf.x, acc[i]);
-            acc[i] = fmaf(wf[2 * j + 1], xf.y, acc[i]);
+        for (int i = 0; i < kD16Tok; ++i) acc[q][i] = 0.f;
+      for (int k0 = lane * 8; k0 < a.K; k0 += 512) {
+        uint4 wv[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            wv[u][q] = (k0 + 256 * u < a.K) ? *reinterpret_cast<const uint4*>(wrow[q] + k0 + 256 * u)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int k = k0 + 256 * u;
+          if (k >= a.K) break;
+#pragma unroll
+          for (int i = 0; i < kD16Tok; ++i) {
+            if (i >= ntok) break;
+            const uint4 xv = *reinterpret_cast<const uint4*>(a.x16 + xr[i] * a.K + k);
+            const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+            float xf[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xx[j]));
+              xf[2 * j] = f.x;
+              xf[2 * j + 1] = f.y;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t ww[4] = {wv[u][q].x, wv[u][q].y, wv[u][q].z, wv[u][q].w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                acc[q][i] = fmaf(__uint_as_float(ww[j] << 16), xf[2 * j], acc[q][i]);
+                acc[q][i] = fmaf(__uint_as_float(ww[j] & 0xFFFF0000u), xf[2 * j + 1], acc[q][i]);
+              }
+            }
           }
         }
       }
 #pragma unroll
-      for (int i = 0; i < kD16Tok; ++i) {
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
-      }
+        for (int i = 0; i < kD16Tok; ++i) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc[q][i] += __shfl_xor_sync(0xFFFFFFFFu, acc[q][i], o);
+        }
       if (lane == 0)
 #pragma unroll
-        for (int i = 0; i < kD16Tok; ++i) red[r][i] = acc[i];
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int i = 0; i < kD16Tok; ++i) red[warp * (kD16Rows / 8) + rg * 4 + q][i] = acc[q][i];
     }
     __syncthreads();
     if (kEpi == kEpiSwiglu) {

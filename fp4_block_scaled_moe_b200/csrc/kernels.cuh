@@ -201,7 +201,7 @@ fp4_status launch_bs(const BsArgs& a, int T, cudaStream_t st);
 fp4_status launch_route_split(const float* logits, int T, int E, int k, const uint16_t* x, int H, int ntok_cap,
                               int32_t* ids, float* gw, int32_t* counts, int32_t* offsets, int32_t* perm,
                               int32_t* inv, uint8_t* q, uint8_t* atoms, cudaStream_t st);
-fp4_status launch_split_x(const uint16_t* x, const int32_t* perm, const int32_t* counts, const int32_t* offsets,
+fp4_status launch_split_x(const uint16_t* x, const int32_t* inv, const int32_t* counts, const int32_t* offsets,
                           int E, int k, int P, int H, int ntok_cap, uint8_t* q, uint8_t* atoms, cudaStream_t st);
 
 // NVFP4 expert GEMMs on the tensor cores (kind::f16, weights widened to f16 on chip).

@@ -322,7 +322,7 @@ fp4_status moe_forward_impl(const fp4_moe_weights* w, const void* x_bf16, const 
       FP4_TRY(launch_route_split(ra.logits, T, E, k, static_cast<const uint16_t*>(x_bf16), H, cap, ra.ids, ra.gw,
                                  ra.counts, ra.offsets, ra.perm, ra.inv, xq, xs, st));
     else
-      FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.perm, ra.counts, ra.offsets, E, k, P, H, cap,
+      FP4_TRY(launch_split_x(static_cast<const uint16_t*>(x_bf16), ra.inv, ra.counts, ra.offsets, E, k, P, H, cap,
                              xq, xs, st));
     BsArgs g{};
     g.epi = kEpiSwiglu;
