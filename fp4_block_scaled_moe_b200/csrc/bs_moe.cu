@@ -105,6 +105,17 @@ __device__ __forceinline__ uint32_t e4m3_rn(float y, float& back) {
   return q;
 }
 
+// Two at once: E4M3 bytes of y0 (low byte) and y1 (high byte), and their exact values
+__device__ __forceinline__ uint32_t e4m3x2_rn(float y0, float y1, float& back0, float& back1) {
+  uint16_t pair;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(y1), "f"(y0));
+  uint32_t h2;
+  asm("{\n .reg .b16 lo;\n cvt.u16.u32 lo, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}" : "=r"(h2) : "r"(static_cast<uint32_t>(pair)));
+  back0 = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
+  back1 = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
+  return pair;
+}
+
 // UE8M0 exponent for a block of E4M3 elements from the bits of its amax (finite, >= 0):
 // the least e with amax * 2^-e <= 448 (E4M3's largest finite value), kept in [-126, 127]
 // so that 2^e and 2^-e are normal floats.  amax in [2^(B-127), 2^(B-126)) for biased
@@ -165,20 +176,21 @@ __device__ __forceinline__ void split_compute(const uint16_t* __restrict__ x, in
   uint32_t* w2 = sp.w2;
   float ramax = 0.f;
 #pragma unroll
-  for (int ii = 0; ii < 32; ++ii) {
-    float b1;
-    const uint32_t c = e4m3_rn(v[ii] * inv1, b1);
+  for (int ii = 0; ii < 32; ii += 2) {
+    float b0, b1;
+    const uint32_t c = e4m3x2_rn(v[ii] * inv1, v[ii + 1] * inv1, b0, b1);
     if ((ii & 3) == 0) w1[ii >> 2] = 0;
     w1[ii >> 2] |= c << (8 * (ii & 3));
-    v[ii] -= b1 * up1;
-    ramax = fmaxf(ramax, fabsf(v[ii]));
+    v[ii] -= b0 * up1;
+    v[ii + 1] -= b1 * up1;
+    ramax = fmaxf(ramax, fmaxf(fabsf(v[ii]), fabsf(v[ii + 1])));
   }
   const int e2 = e4m3_block_exp(ramax);
   const float inv2 = exp2i(-e2);
 #pragma unroll
-  for (int ii = 0; ii < 32; ++ii) {
-    float b2;
-    const uint32_t c = e4m3_rn(v[ii] * inv2, b2);
+  for (int ii = 0; ii < 32; ii += 2) {
+    float b0, b1;
+    const uint32_t c = e4m3x2_rn(v[ii] * inv2, v[ii + 1] * inv2, b0, b1);
     if ((ii & 3) == 0) w2[ii >> 2] = 0;
     w2[ii >> 2] |= c << (8 * (ii & 3));
   }

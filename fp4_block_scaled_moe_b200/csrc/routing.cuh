@@ -49,12 +49,10 @@ __device__ __forceinline__ void topk_warp_n(const float* __restrict__ lg, int E,
         if (key[j] > best || (key[j] == best && e < best_e)) { best = key[j]; best_e = e; }
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-      const int oe = __shfl_xor_sync(0xFFFFFFFFu, best_e, o);
-      if (ob > best || (ob == best && oe < best_e)) { best = ob; best_e = oe; }
-    }
+    // the warp's largest key, then the lowest expert holding it (two warp reductions)
+    const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, best);
+    best_e = __reduce_min_sync(0xFFFFFFFFu, best == wmax ? best_e : 0x7FFFFFFF);
+    best = wmax;
     if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
     const float l = key_value(best);                 // the logit itself (-0 read as +0)
     if (r == 0) m = l;
