@@ -514,7 +514,7 @@ def moe_roofline(cfg, counts, extra_gu, kern_ms, tensor, peaks):
                                      else "fallback 1590 TFLOP/s bf16 (of fallback)"),
                      "frac_of_sustained": (ach / peaks["bf16_tflops_sustained"])
                      if ach and "bf16_tflops_sustained" in peaks else None,
-                     "frac_of_fp4_measured": (ach / bs["mxfp4"]) if ach and bs.get("mxfp4") else None,
+                     "frac_of_fp4_measured": (ach / bs[cfg.fmt]) if ach and bs.get(cfg.fmt) else None,
                      "frac_of_mxfp8_measured": (ach / bs["mxfp8"]) if ach and bs.get("mxfp8") else None,
                      "frac_of_fp4_nominal_9000": (ach / 9000.0) if ach else None,
                      "flops_per_launch": int(flops)})
