@@ -3,6 +3,8 @@ every replay of a captured CUDA graph give identical y bits.  Work units are han
 CTAs from an atomic counter, so which CTA runs a unit varies from call to call; each
 unit owns its output rows and sums its K in a fixed order, and the combine adds the k
 slots of a token in j order, so the bits do not depend on that schedule."""
+from dataclasses import replace
+
 import numpy as np
 import pytest
 import torch
@@ -23,6 +25,8 @@ _CASES = [
     ("c3_small_nvfp4_tensor", C.small(C.MOE_C3), 2, False),
     ("c3_full_nvfp4_tensor", C.MOE_C3, 2, True),
     ("c4nv_full_tensor", C.MOE_C4_NV, 0, True),
+    ("nvfp4_t48_gemv_16_token_units", replace(C.MOE_C3, name="nvfp4_t48_e64_k4_zipf", T=48, E=64, H=512, I=256, k=4),
+     1, False),
 ]
 
 

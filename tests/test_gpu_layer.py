@@ -143,6 +143,16 @@ def test_moe_small(cfg):
     _moe_case(cfg)
 
 
+# NVFP4 GEMV units of up to 16 tokens (T >= 32 and T k >= 2E): the Zipf-skewed router puts
+# 17-48 tokens on four experts (two or three 16-token units each), 9-16 on one and 1-8 on
+# five, so full, partial and single-tile units all run
+@pytest.mark.parametrize("variant", [0, 1], ids=["auto", "gemv"])
+def test_moe_nvfp4_sixteen_token_units(variant):
+    from dataclasses import replace
+    cfg = replace(C.MOE_C3, name="nvfp4_t48_e64_k4_zipf", T=48, E=64, H=512, I=256, k=4)
+    _moe_case(cfg, variant=variant)
+
+
 @pytest.mark.parametrize("cfg", [C.small(C.MOE_C2_MIXED), C.MOE_C2_MIXED], ids=["small", "full"])
 def test_moe_mixed_format_buffer(cfg):
     """A fused buffer holding MXFP4 experts and bf16 experts (kept out of quantisation),
