@@ -232,10 +232,10 @@ typedef struct fp4_moe_weights {
   const int32_t* dn_rowptr;
   const int32_t* dn_col;
   const uint16_t* dn_val;
-  /* Expert-GEMM kernels: 0 = chosen per call (tensor cores when T*k >= 4E, i.e. four
-   * or more tokens per expert on average, and for MXFP4 also whenever gu_mma_scales /
-   * dn_mma_scales are given; else the CUDA-core GEMV), 1 = CUDA-core grouped GEMV,
-   * 2 = tensor-core GEMM (MXFP4: block-scaled kind::mxf8f6f4; NVFP4: weights widened to
+  /* Expert-GEMM kernels: 0 = chosen per call (MXFP4: tensor cores when T*k >= 4E, i.e.
+   * four or more tokens per expert on average, or whenever gu_mma_scales / dn_mma_scales
+   * are given; NVFP4: tensor cores when T*k >= 64E; else the CUDA-core GEMV), 1 = CUDA-core
+   * grouped GEMV, 2 = tensor-core GEMM (MXFP4: block-scaled kind::mxf8f6f4; NVFP4: weights widened to
    * f16 on chip, kind::f16; FP4_ERR_UNSUPPORTED for CB4 or unsupported shapes).
    * Any other value is FP4_ERR_INVALID_ARG. */
   int32_t kernel_variant;

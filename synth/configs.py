@@ -94,7 +94,11 @@ MOE_C3_PROFILE = MoEConfig("moe_nvfp4_decode_e64_h6144_i2048_k8_t16_zipf", "nvfp
                            k=8, zipf_bias=True, outliers=(0.003, 10.0, 49.0))
 MOE_C4NV_PROFILE = MoEConfig("moe_nvfp4_prefill_e64_h6144_i2048_k8_t2048", "nvfp4", T=2048, E=64, H=6144,
                              I=2048, k=8)
-PROFILE = {c.name: c for c in (MOE_C4_PROFILE, MOE_C3_PROFILE, MOE_C4NV_PROFILE)}
+# The NVFP4 decode layer at a quarter of the experts with all 64 tokens (units of up to
+# 16 tokens, as in the full layer): 1.36 GB of weights.
+MOE_C3_PROFILE_T64 = MoEConfig("moe_nvfp4_decode_e64_h6144_i2048_k8_t64_zipf", "nvfp4", T=64, E=64, H=6144,
+                               I=2048, k=8, zipf_bias=True, outliers=(0.003, 10.0, 49.0))
+PROFILE = {c.name: c for c in (MOE_C4_PROFILE, MOE_C3_PROFILE, MOE_C4NV_PROFILE, MOE_C3_PROFILE_T64)}
 
 
 def small(cfg):
