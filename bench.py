@@ -5,11 +5,16 @@
 Default (--config all): every workload on each GPU, reported as ONE JSON line. The
 top-level keys are the headline workload, the largest single-GPU configuration: the
 MXFP4 MoE prefill layer (8192 bf16 tokens, 256 experts, hidden 6144, expert
-intermediate 2048, top-8). "workloads" holds the same record for the other four:
+intermediate 2048, top-8). "workloads" holds the same record for the other seven:
 the dense MXFP4 W4A16 linear layer (16 x 2048 x 2048), the MXFP4 decode layer (64
 experts, hidden 2048, intermediate 768, top-8, 16 tokens), the NVFP4 decode layer
-(256 experts, hidden 6144, intermediate 2048, 64 tokens, Zipf-skewed router) and the
-CB4 codebook-plus-outlier decode layer (the MXFP4 decode layer's dimensions).
+(256 experts, hidden 6144, intermediate 2048, 64 tokens, Zipf-skewed router), the CB4
+codebook-plus-outlier decode layer (the MXFP4 decode layer's dimensions), the NVFP4
+prefill layer (the MXFP4 prefill layer's dimensions), the V2a shared-library decode layer
+and a mixed buffer of MXFP4 and bf16 experts (both at the MXFP4 decode layer's
+dimensions).  Each record carries its roofline (dominant kernel's device time per launch,
+algorithmic bytes or flops, DRAM traffic from the committed ncu summary of the same
+kernel sources), e2e, clocks, launch count and CPU-oracle baseline.
 
 One step = one full layer call (router, gate_up + fused SwiGLU-with-clamp, down,
 weighted combine; for the linear layer one y = x W^T) on device-resident inputs,
