@@ -33,3 +33,20 @@ def test_prefill_flops_and_units():
     assert unit == "TFLOP/s" and abs(work - 4.948e12 / 1e12) < 1e-3
     work, unit = bench.work_per_step(C.MOE_C2, np.ones(C.MOE_C2.E))
     assert unit == "GB/s"
+
+
+def test_mixed_gemv_roofline_counts_only_the_mxfp4_experts():
+    """In a mixed buffer the GEMV reads the routed MXFP4 experts; the bf16 experts run in
+    their own kernel, so the GEMV's roofline bytes leave them out (the layer's bytes keep
+    them)."""
+    cfg = C.MOE_C2_MIXED
+    counts = np.zeros(cfg.E, dtype=np.int64)
+    bf = list(cfg.bf16_experts)
+    counts[[0, 1, 2] + bf[:2]] = 1                     # three MXFP4 experts and two bf16 ones
+    r = bench.moe_roofline(cfg, counts, None, {"gate_up": 1.0, "down": 1.0}, False, {})
+    gu = bench.per_expert_bytes(cfg)[1]
+    P = cfg.T * cfg.k
+    assert r["bytes_per_launch"] == 3 * gu + cfg.T * cfg.H * 2 + P * cfg.I * 2
+    # the same routing in a pure MXFP4 buffer counts all five
+    r2 = bench.moe_roofline(C.MOE_C2, counts, None, {"gate_up": 1.0, "down": 1.0}, False, {})
+    assert r2["bytes_per_launch"] == 5 * gu + cfg.T * cfg.H * 2 + P * cfg.I * 2
