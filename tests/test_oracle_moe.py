@@ -133,3 +133,29 @@ def test_moe_token_subset_matches_full():
     full = M.moe_forward(x, ids, w, bank)
     sub = M.moe_forward(x, ids, w, bank, tokens=[7, 2, 5])
     assert np.allclose(sub, full[[7, 2, 5]], rtol=1e-13, atol=1e-13)
+
+
+def test_mixed_bank_reduces_to_its_parts():
+    """A mixed-format bank ("The gate that missed by 0.0202 pp", "A fused tensor with two
+    dtypes in it") is, expert by expert, the MXFP4 bank for the quantised experts and the
+    bf16-rounded weights for the excluded ones: a single excluded expert gives the textbook
+    FFN on bf16 weights, and no excluded expert gives the MXFP4 bank."""
+    rng = np.random.default_rng(17)
+    E, H, I, T = 3, 64, 32, 4
+    gu = rng.normal(0, 0.05, (E, 2 * I, H)).astype(np.float32)
+    dn = rng.normal(0, 0.05, (E, H, I)).astype(np.float32)
+    draw = lambda which, e: gu[e] if which == "gu" else dn[e]   # noqa: E731
+    x = rng.normal(size=(T, H))
+    mixed = M.LazyExpertBank("mixed", E, H, I, draw, bf16_experts=(1,))
+    mx = M.LazyExpertBank("mxfp4", E, H, I, draw)
+    ids = np.full((T, 1), 1, np.int32)
+    w = np.ones((T, 1))
+    y_bf16 = M.moe_forward(x, ids, w, mixed)
+    ref = _ffn(x, F.round_to_bf16(gu[1].astype(np.float64)), F.round_to_bf16(dn[1].astype(np.float64)), I)
+    assert np.allclose(y_bf16, ref, rtol=1e-13, atol=1e-13)
+    for e in (0, 2):
+        ids = np.full((T, 1), e, np.int32)
+        assert np.array_equal(M.moe_forward(x, ids, w, mixed), M.moe_forward(x, ids, w, mx))
+    # the bf16 expert differs from its MXFP4 quantisation (the formats really differ)
+    ids = np.full((T, 1), 1, np.int32)
+    assert not np.allclose(M.moe_forward(x, ids, w, mixed), M.moe_forward(x, ids, w, mx), rtol=1e-3)
