@@ -34,9 +34,7 @@ int moe_variant(const fp4_moe_weights* w, int32_t T, int32_t k) {
   if (w->kernel_variant == kVarTensor) return kVarTensor;
   if (w->kernel_variant == kVarGemv) return kVarGemv;
   // MXFP4: tensor cores when the scale atoms come with the weights, or when the call has
-  // enough tokens per expert to amortise re-laying them in the workspace.  NVFP4: tensor
-  // cores only for the latter (at decode sizes the weight-widening tensor-core kernel
-  // streams slower than the CUDA-core GEMV).
+  // enough tokens per expert to amortise re-laying them in the workspace.
   const bool prepared = w->gu_mma_scales != nullptr && w->dn_mma_scales != nullptr;
   const bool many = static_cast<int64_t>(T) * k >= 4 * static_cast<int64_t>(w->num_experts);
   // NVFP4 widens its weights on chip before the tensor cores; measured on the NVFP4 decode

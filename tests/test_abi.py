@@ -186,3 +186,16 @@ def test_linear_named_refusals():
     assert lin(L.FP4_MXFP4, 4, 256, 65) == 5
     assert lin(L.FP4_MXFP4, 4, 1 << 40, 64) == 3
     assert lin(L.FP4_MXFP4, 4, 256, 64, ws=None) == 6
+
+
+def test_automatic_expert_kernels_follow_the_measured_crossovers():
+    """kernel_variant 0: MXFP4 takes the tensor cores from 4 routed pairs per expert (or
+    with prepared scale atoms), NVFP4 from 64 (below, the GEMV with 16-token units is
+    faster than widening the weights on chip)."""
+    lib = L.load()
+    ek = lambda w, T, k: lib.moe_fp4_expert_kernels(ctypes.byref(w), T, k)   # noqa: E731
+    nv, mx = _weights(fmt=L.FP4_NVFP4, E=8), _weights(fmt=L.FP4_MXFP4, E=8)
+    assert ek(nv, 63, 8) == 1 and ek(nv, 64, 8) == 2
+    assert ek(mx, 3, 8) == 1 and ek(mx, 4, 8) == 2
+    mx.gu_mma_scales = mx.dn_mma_scales = 0x10000
+    assert ek(mx, 1, 8) == 2
