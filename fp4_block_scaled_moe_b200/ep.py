@@ -32,20 +32,27 @@ def expert_range(rank: int, world: int, E: int):
 
 def shard(weights: MoEWeights, rank: int, world: int) -> MoEWeights:
     """The experts of ``rank`` cut from a full layer's weights (copies, contiguous). The
-    CB4 outlier CSR, one per fused matrix over E * rows rows, is cut to the local rows and
-    its row pointers re-based."""
+    CB4 / V2a outlier CSR, one per fused matrix over E * rows rows, is cut to the local rows
+    and its row pointers re-based; CB4 codebooks are cut by rows, V2a libraries (one per
+    expert matrix) by expert.  Mixed-format buffers are refused (their byte offsets would
+    need re-basing, which is not implemented)."""
     if weights.local_experts not in (0, weights.E) or weights.expert_begin != 0:
         raise ValueError("shard() takes a full layer")
+    if weights.expert_format is not None:
+        raise ValueError("shard() does not cut mixed-format buffers")
     b, n = expert_range(rank, world, weights.E)
     cut = {}
     per_expert = ("gu_codes", "gu_scales", "dn_codes", "dn_scales", "gu_tscale", "dn_tscale")
     for name in per_expert:
         t = getattr(weights, name)
         cut[name] = None if t is None else t[b:b + n].contiguous()
-    if weights.fmt == "cb4":
+    if weights.fmt in ("cb4", "v2a"):
         for pre, rows in (("gu", 2 * weights.I), ("dn", weights.H)):
             cb = getattr(weights, pre + "_cb")
-            cut[pre + "_cb"] = cb.view(weights.E, rows, *cb.shape[1:])[b:b + n].reshape(n * rows, *cb.shape[1:]).contiguous()
+            if weights.fmt == "cb4":
+                cut[pre + "_cb"] = cb.view(weights.E, rows, *cb.shape[1:])[b:b + n].reshape(n * rows, *cb.shape[1:]).contiguous()
+            else:
+                cut[pre + "_cb"] = cb[b:b + n].contiguous()
             rp = getattr(weights, pre + "_rowptr")
             r0, r1 = b * rows, (b + n) * rows
             lo = rp[r0:r0 + 1]

@@ -67,6 +67,32 @@ def test_shard_cuts_cb4_layer_and_rebases_csr():
             assert torch.equal(val.long(), torch.repeat_interleave(torch.arange(b, b + n), torch.arange(b, b + n) + 1))
 
 
+def test_shard_cuts_v2a_libraries_by_expert():
+    """V2a: the group records cut like scales, the per-expert libraries by expert, the CSR
+    like CB4's."""
+    w = _cb4_weights()
+    E, I, H = w.E, w.I, w.H
+    lib = lambda: torch.arange(E, dtype=torch.int16).view(E, 1, 1).expand(E, 32, 16).contiguous()   # noqa: E731
+    v = MoEWeights("v2a", E, H, I, w.gu_codes, w.gu_codes.clone(), w.dn_codes, w.dn_codes.clone(), None, None, 7.0,
+                   gu_cb=lib(), gu_rowptr=w.gu_rowptr, gu_col=w.gu_col, gu_val=w.gu_val,
+                   dn_cb=lib(), dn_rowptr=w.dn_rowptr, dn_col=w.dn_col, dn_val=w.dn_val)
+    for rank, world in ((0, 2), (1, 3), (3, 4)):
+        s = ep.shard(v, rank, world)
+        b, n = ep.expert_range(rank, world, E)
+        assert s.gu_cb.shape == (n, 32, 16) and torch.equal(s.dn_cb[:, 0, 0].long(), torch.arange(b, b + n))
+        assert torch.equal(s.gu_scales[:, 0, 0].long(), torch.arange(b, b + n))
+        rp = s.gu_rowptr
+        assert rp.shape[0] == n * 2 * I + 1 and int(rp[0]) == 0 and int(rp[-1]) == s.gu_val.shape[0]
+
+
+def test_shard_refuses_mixed_buffers():
+    w = _cb4_weights()
+    m = MoEWeights("mxfp4", w.E, w.H, w.I, w.gu_codes, w.gu_codes, w.dn_codes, w.dn_codes,
+                   expert_format=torch.zeros(w.E, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        ep.shard(m, 0, 2)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
